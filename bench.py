@@ -1,0 +1,441 @@
+"""Benchmark of the microscaled linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3|c2|c4|c1]
+                    [--impl mxq|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+for NVFP4, activation amax -> NVFP4 quantisation -> block-scaled GEMM with the
+bias epilogue; for MXFP8, quantisation -> GEMM.  Weights are quantised once,
+before timing (offline, as the method prescribes).  The default workload is
+the NVFP4 MLP-up layer M=4608, K=3072, N=12288 (bias, 0.1 % outlier
+channels).  The metric is TFLOP/s of the GEMM (2MNK per step) including the
+activation quantisation.
+
+Timing: W untimed warm-up steps; K timed steps bracketed by a barrier and
+torch.cuda.synchronize(); CUDA events on the launching stream; max over
+ranks.  Each step uses one of several rotating buffer sets whose total size
+is well above the 126 MB L2, so no step starts with its inputs in L2.  Under
+torchrun each rank runs an independent replica (weak scaling: no data-path
+collective; the path does not shard).
+
+--impl reference times the CPU oracle (the plain numpy restatement of the
+method) on a bounded sample of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "block-scaled GEMM TFLOPS incl. act quant; % of dense FP4/FP8 peak"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+# Dense tensor peaks (TFLOP/s) for the roofline: the measured cuBLAS bf16
+# figure of this machine pool times the nominal FP4:BF16 (4x) / FP8:BF16 (2x)
+# ratio of B200; fallback numbers when no measurement file is present.
+NOMINAL_RATIO = {"nvfp4": 4.0, "mxfp8": 2.0, "bf16": 1.0}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(bf16=float(p["bf16_tflops"]), bf16_sustained=float(p["bf16_tflops_sustained"]),
+                    hbm=float(p["hbm_gbs"]), source="measured")
+    except Exception:
+        return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+def _nvml_id(local_rank: int):
+    """NVML index (int) or UUID (str) of this rank's GPU."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if not vis:
+        return local_rank
+    entry = vis.split(",")[local_rank].strip()
+    return int(entry) if entry.isdigit() else entry
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device, period_s: float = 0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = (pynvml.nvmlDeviceGetHandleByIndex(device) if isinstance(device, int)
+                       else pynvml.nvmlDeviceGetHandleByUUID(device))
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                break
+            time.sleep(self.period)
+
+    def start(self):
+        if self._h is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if self._h is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ the GPU arm
+def run_gpu(args, rank, world, local_rank):
+    import fp8_gemm_diffusion_b200 as mxq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    case = workloads.make_case(args.workload)
+    fmt = case.fmt
+    M, K, N = case.M, case.K, case.N
+    flops = 2.0 * M * N * K
+    stream = torch.cuda.current_stream(dev)
+
+    # one prepared weight, then per-set copies of everything a step touches
+    W = case.W.to(dev)
+    bias = case.bias.to(dev) if case.bias is not None else None
+    base_w = mxq.Weight(W, bias, fmt=fmt)
+    per_set = (M * K * 2 + mxq.weight_storage_bytes(N, K, fmt) + M * N * 2
+               + mxq.linear_workspace_bytes(M, K, fmt))
+    nsets = max(2, int(np.ceil(3 * L2_BYTES / per_set)))
+    A0 = case.A.to(dev)
+    sets = []
+    for _ in range(nsets):
+        storage = base_w.storage.clone()
+        h = mxq.mxq_weight.from_buffer_copy(base_w.handle)
+        off = storage.data_ptr() - base_w.storage.data_ptr()
+        h.codes += off
+        h.sf += off
+        if h.g_dev:
+            h.g_dev += off
+            h.amax_dev += off
+        ws_bytes = mxq.linear_workspace_bytes(M, K, fmt)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        sets.append(dict(x=A0.clone(), storage=storage, w=h,
+                         y=torch.empty(M, N, dtype=torch.bfloat16, device=dev), ws=ws,
+                         ws_bytes=ws_bytes,
+                         amax=ws[0:4].view(torch.float32), g=ws[4:8].view(torch.float32)))
+    torch.cuda.synchronize()
+    lay_codes = 256
+    lay_sf = lay_codes + (mxq.codes_bytes(M, K, fmt) + 255) // 256 * 256
+
+    def step(i, ev=None):
+        s = sets[i % nsets]
+        ws = s["ws"]
+        codes = ws[lay_codes:]
+        sf = ws[lay_sf:]
+        h = s["w"]
+        if ev is not None:
+            ev[0].record(stream)
+        if fmt == "nvfp4":
+            mxq.amax(s["x"], s["amax"], stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+            mxq.quantize_nvfp4(s["x"], s["amax"], codes, sf, s["g"], stream=stream)
+        else:
+            if ev is not None:
+                ev[1].record(stream)
+            mxq.quantize_mxfp8(s["x"], codes, sf, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        mxq.gemm_blockscaled(fmt, M, N, K, codes, sf, s["g"] if fmt == "nvfp4" else None,
+                             h.codes, h.sf, h.g_dev if fmt == "nvfp4" else None,
+                             bias, s["y"], stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    launches_per_step = 3 if fmt == "nvfp4" else 2
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+    # warm-up
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if mxq.get_device_error() != mxq.OK:
+        raise RuntimeError("device-side timeout during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(_nvml_id(local_rank))
+    if dist:
+        tdist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    if dist:
+        tdist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    amax_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    quant_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    gemm_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    if mxq.get_device_error() != mxq.OK:
+        raise RuntimeError("device-side timeout during the timed steps")
+    if dist:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end through the public call with host buffers
+    e2e = run_e2e(mxq, case, base_w, dev, stream, args, dist)
+
+    peaks = _peaks()
+    peak = peaks["bf16"] * NOMINAL_RATIO[fmt]
+    gemm_avg_s = float(np.mean(gemm_ms)) * 1e-3
+    achieved = flops / gemm_avg_s / 1e12
+    value = world * args.steps * flops / (total_ms * 1e-3) / 1e12
+    qbytes = (M * K * 2 + M * K // (2 if fmt == "nvfp4" else 1)
+              + mxq.sf_bytes(M, K, fmt))
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e2m1+e4m3 (nvfp4), fp32 accumulate, bf16 out" if fmt == "nvfp4"
+        else "e4m3+e8m0 (mxfp8), fp32 accumulate, bf16 out",
+        "data": "synthetic (seeded, FLUX-shaped; random-init weights)",
+        "config": {
+            "workload": case.name, "format": fmt, "M": M, "K": K, "N": N,
+            "bias": case.bias is not None, "parallelism": f"replicas x{world}",
+            "l2": f"rotating {nsets} buffer sets ({nsets * per_set / 2**20:.0f} MiB > 126 MiB L2)",
+        },
+        "fraction_of_dense_peak": {
+            "nominal": round(value / ({"nvfp4": 9000.0, "mxfp8": 4500.0}[fmt]), 4),
+            "nominal_peak_tflops": {"nvfp4": 9000.0, "mxfp8": 4500.0}[fmt],
+        },
+        "kernels_ms": {
+            "amax": round(float(np.mean(amax_ms)), 5),
+            "quantize": round(float(np.mean(quant_ms)), 5),
+            "gemm": round(float(np.mean(gemm_ms)), 5),
+        },
+        "quantize_gbs": round(qbytes / (float(np.mean(quant_ms)) * 1e-3) / 1e9, 1),
+        "roofline": {
+            "kernel": f"gemm_kernel<{fmt}>",
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": round(peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} TFLOP/s x "
+                           f"{NOMINAL_RATIO[fmt]:g} (nominal {fmt}:bf16 ratio)",
+            "traffic": None,
+        },
+        "clocks": sampler.summary(),
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    return result
+
+
+def run_e2e(mxq, case, base_w, dev, stream, args, dist):
+    """Same metric through mxq_linear with pinned host input and output:
+    each step copies A host->device, runs the layer, copies Y device->host."""
+    M, K, N = case.M, case.K, case.N
+    fmt = case.fmt
+    x_host = case.A.pin_memory()
+    y_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    y_dev = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    ws_bytes = mxq.linear_workspace_bytes(M, K, fmt)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    steps = max(3, min(args.steps, 20))
+
+    def one():
+        x_dev.copy_(x_host, non_blocking=True)
+        mxq.linear(base_w.handle, x_dev, M, y_dev, ws, ws_bytes, stream=stream)
+        y_host.copy_(y_dev, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    if dist:
+        import torch.distributed as tdist
+        tdist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms = float(t.item())
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    flops = 2.0 * M * N * K
+    return {"value": round(world * steps * flops / (ms * 1e-3) / 1e12, 3), "unit": UNIT,
+            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "steps": steps}
+
+
+# ------------------------------------------------------------- CPU oracle
+def run_oracle_sample(workload: str, budget_s: float = 12.0):
+    """Time the oracle (as it stands) on a bounded sample of the workload:
+    the activation's global amax, then quantisation + float64 GEMM of row
+    chunks until the time budget is spent.  Weight quantisation is offline
+    (done before timing), as on the GPU."""
+    from oracle import gemm as G
+    from oracle import quant as Q
+
+    case = workloads.make_case(workload)
+    fmt = case.fmt
+    M, K, N = case.M, case.K, case.N
+    if fmt == "nvfp4":
+        qw = Q.quantize_nvfp4(case.W)
+        Wd = Q.dequant_nvfp4(qw["codes"], qw["sf"], qw["g"])
+    else:
+        qw = Q.quantize_mxfp8(case.W)
+        Wd = Q.dequant_mxfp8(qw["codes"], qw["sf"])
+    chunk = 64
+    rows_done = 0
+    t0 = time.perf_counter()
+    amax = Q.amax(case.A) if fmt == "nvfp4" else None
+    while time.perf_counter() - t0 < budget_s and rows_done < M:
+        r0 = rows_done
+        a = case.A[r0:r0 + chunk]
+        if fmt == "nvfp4":
+            qa = Q.quantize_nvfp4(a, global_amax=amax)
+            Ad = Q.dequant_nvfp4(qa["codes"], qa["sf"], qa["g"])
+        else:
+            qa = Q.quantize_mxfp8(a)
+            Ad = Q.dequant_mxfp8(qa["codes"], qa["sf"])
+        G.linear_ref(Ad, Wd, case.bias)
+        rows_done += a.shape[0]
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows_done * N * K
+    try:
+        threads = len(os.sched_getaffinity(0))
+    except Exception:
+        threads = os.cpu_count()
+    return {
+        "value": round(flops / dt / 1e12, 6),
+        "unit": UNIT,
+        "cores": threads,
+        "kind": "oracle",
+        "sample": f"{rows_done} of {M} rows of {case.name}: amax of the full activation, "
+                  f"then {fmt} quantisation + float64 GEMM (Y and sum|ab|) in {chunk}-row "
+                  f"chunks, {dt:.1f} s",
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4"])
+    ap.add_argument("--impl", default="mxq", choices=["mxq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        # the CPU oracle on the host cores: rank 0 only, a few bounded samples
+        if rank != 0:
+            return 0
+        steps = max(1, min(args.steps, 3))
+        per_step, sample = [], None
+        for _ in range(steps):
+            sample = run_oracle_sample(args.workload, budget_s=4.0)
+            per_step.append(sample["value"])
+        value = float(np.median(per_step))
+        out = {
+            "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": steps, "warmup": 0,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 quantisation, f64 GEMM (CPU oracle)", "data": "synthetic",
+            "config": {"workload": workloads.CASE_NAMES[args.workload]},
+            "cpu_baseline": {"value": value, "unit": UNIT, "kind": sample["kind"],
+                             "cores": sample["cores"], "sample": sample["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(out))
+        return 0
+
+    dist = world > 1
+    if dist:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local_rank))
+    try:
+        result = run_gpu(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = run_oracle_sample(args.workload)
+        if rank == 0:
+            print(json.dumps(result))
+    finally:
+        if dist:
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

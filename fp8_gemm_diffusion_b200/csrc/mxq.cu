@@ -1,0 +1,517 @@
+// mxq.cu - the C ABI (include/mxq.h): argument checks, dispatch, launches.
+//
+// One translation unit holds every kernel (quant.cuh, gemm.cuh) so that they
+// share the device error word.  Built with nvcc for sm_100a only, without
+// fast-math (the quantisers must round exactly like the definition).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mxq.h"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+thread_local int t_last_cuda_error = 0;
+
+inline int64_t pad_to(int64_t n, int64_t m) { return (n + m - 1) / m * m; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+mxq_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return MXQ_ERR_CUDA;
+}
+
+// ------------------------------------------------------- device properties
+struct DeviceInfo {
+  std::atomic<int> state{0};  // 0 unknown, 1 supported, 2 unsupported
+  int sms = 0;
+  std::atomic<uint32_t> smem_attr_set{0};  // bit per GEMM instantiation
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+mxq_status current_device(int* dev_out, int* sms_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    t_last_cuda_error = static_cast<int>(e);
+    cudaGetLastError();
+    return MXQ_ERR_ARCH;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return MXQ_ERR_ARCH;
+  DeviceInfo& d = g_dev[dev];
+  int st = d.state.load(std::memory_order_acquire);
+  if (st == 0) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    st = d.state.load(std::memory_order_relaxed);
+    if (st == 0) {
+      int major = 0, minor = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MXQ_ERR_ARCH;
+      }
+      d.sms = sms;
+      st = (major == 10 && minor == 0) ? 1 : 2;  // sm_100a code runs on compute capability 10.0
+      d.state.store(st, std::memory_order_release);
+    }
+  }
+  if (st != 1) return MXQ_ERR_ARCH;
+  *dev_out = dev;
+  if (sms_out) *sms_out = d.sms;
+  return MXQ_OK;
+}
+
+// ------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+mxq_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    } else {
+      cudaGetLastError();
+    }
+  });
+  return g_encode ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+// 2-D row-major tensor [outer][inner] with a row stride in bytes.
+mxq_status tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner,
+                   uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                   uint32_t box_outer, CUtensorMapSwizzle swz) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda_error = static_cast<int>(r);
+    return MXQ_ERR_CUDA;
+  }
+  return MXQ_OK;
+}
+
+int quant_grid(int64_t vectors, int sms) {
+  const int64_t per_block = static_cast<int64_t>(mxq::kQuantThreads) * mxq::kQuantUnroll;
+  int64_t g = (vectors + per_block - 1) / per_block;
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+mxq_status check_bf16_matrix(const void* x, int64_t rows, int64_t k, int64_t ld) {
+  if (rows < 0 || k < 0) return MXQ_ERR_INVALID_ARG;
+  if (rows > 0 && k > 0 && x == nullptr) return MXQ_ERR_INVALID_ARG;
+  if (ld < k || ld < 1) return MXQ_ERR_INVALID_ARG;
+  if (ld % 8 != 0) return MXQ_ERR_ALIGNMENT;
+  if (!aligned16(x)) return MXQ_ERR_ALIGNMENT;
+  if (rows > INT32_MAX || k > INT32_MAX) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  return MXQ_OK;
+}
+
+// ----------------------------------------------------------------- launches
+mxq_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ld, float* amax,
+                       cudaStream_t s, int sms) {
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (rows == 0 || k == 0) return MXQ_OK;
+  const int64_t vectors = rows * (k / 8);
+  mxq::amax_kernel<<<quant_grid(vectors, sms), mxq::kQuantThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), rows, k, ld, amax);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
+}
+
+mxq_status launch_quant_nvfp4(const void* x, int64_t rows, int64_t k, int64_t ld,
+                              const float* amax, uint8_t* codes, uint8_t* sf, float* g,
+                              cudaStream_t s, int sms) {
+  const int64_t vectors = rows * (k / 8);
+  mxq::quantize_nvfp4_kernel<<<quant_grid(vectors, sms), mxq::kQuantThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), rows, k, ld, amax, codes, sf, g);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
+}
+
+mxq_status launch_quant_mxfp8(const void* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
+                              uint8_t* sf, cudaStream_t s, int sms) {
+  const int64_t vectors = rows * (k / 8);
+  mxq::quantize_mxfp8_kernel<<<quant_grid(vectors, sms), mxq::kQuantThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), rows, k, ld, codes, sf);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
+}
+
+template <mxq::Fmt F, int BN>
+mxq_status launch_gemm_bn(int dev, int sms, int slot, int64_t M, int64_t N, int64_t K,
+                          const void* a, const uint8_t* a_sf, const float* a_g, const void* b,
+                          const uint8_t* b_sf, const float* b_g, const void* bias, void* y,
+                          int64_t ldy, cudaStream_t s) {
+  using C = mxq::GemmCfg<F, BN>;
+  auto kern = mxq::gemm_kernel<F, BN>;
+  const uint32_t bit = 1u << slot;
+  if (!(g_dev[dev].smem_attr_set.load(std::memory_order_acquire) & bit)) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_dev[dev].smem_attr_set.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  CUtensorMap ta, tb, ty;
+  mxq_status st;
+  if (F == mxq::Fmt::BF16) {
+    st = tmap_2d(&ta, a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 64, C::BM,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st == MXQ_OK)
+      st = tmap_2d(&tb, b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, N, K * 2, 64, BN,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    const int64_t row_bytes = F == mxq::Fmt::NVFP4 ? K / 2 : K;
+    st = tmap_2d(&ta, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, row_bytes, M, row_bytes, 128, C::BM,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st == MXQ_OK)
+      st = tmap_2d(&tb, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, row_bytes, N, row_bytes, 128, BN,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  if (st == MXQ_OK)
+    st = tmap_2d(&ty, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, ldy * 2, 32, 32,
+                 CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != MXQ_OK) return st;
+  mxq::GemmArgs args;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.a_sf = a_sf;
+  args.b_sf = b_sf;
+  args.a_g = a_g;
+  args.b_g = b_g;
+  args.bias = static_cast<const __nv_bfloat16*>(bias);
+  const int64_t tiles = ((M + C::BM - 1) / C::BM) * ((N + BN - 1) / BN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, ty, args);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
+}
+
+mxq_status launch_gemm(mxq_format f, int dev, int sms, int64_t M, int64_t N, int64_t K,
+                       const void* a, const uint8_t* a_sf, const float* a_g, const void* b,
+                       const uint8_t* b_sf, const float* b_g, const void* bias, void* y,
+                       int64_t ldy, cudaStream_t s) {
+  switch (f) {
+    case MXQ_NVFP4:
+      if (N % 192 == 0)
+        return launch_gemm_bn<mxq::Fmt::NVFP4, 192>(dev, sms, 0, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                     b_g, bias, y, ldy, s);
+      return launch_gemm_bn<mxq::Fmt::NVFP4, 128>(dev, sms, 1, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                   b_g, bias, y, ldy, s);
+    case MXQ_MXFP8:
+      if (N % 192 == 0)
+        return launch_gemm_bn<mxq::Fmt::MXFP8, 192>(dev, sms, 2, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                     b_g, bias, y, ldy, s);
+      return launch_gemm_bn<mxq::Fmt::MXFP8, 128>(dev, sms, 3, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                   b_g, bias, y, ldy, s);
+    case MXQ_BF16:
+      if (N % 256 == 0)
+        return launch_gemm_bn<mxq::Fmt::BF16, 256>(dev, sms, 4, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                    b_g, bias, y, ldy, s);
+      return launch_gemm_bn<mxq::Fmt::BF16, 128>(dev, sms, 5, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                  b_g, bias, y, ldy, s);
+  }
+  return MXQ_ERR_INVALID_ARG;
+}
+
+bool valid_format(int f) { return f == MXQ_NVFP4 || f == MXQ_MXFP8 || f == MXQ_BF16; }
+
+// Byte layout shared by the activation workspace and weight storage:
+// [0,4) amax, [4,8) g, [256, 256+codes) codes, then the scales (256-aligned).
+struct QuantLayout {
+  size_t codes_off, sf_off, total;
+};
+QuantLayout quant_layout(int64_t rows, int64_t k, mxq_format f) {
+  QuantLayout l;
+  l.codes_off = 256;
+  l.sf_off = l.codes_off + static_cast<size_t>(pad_to(mxq_codes_bytes(rows, k, f), 256));
+  l.total = l.sf_off + static_cast<size_t>(pad_to(mxq_sf_bytes(rows, k, f), 256));
+  return l;
+}
+
+}  // namespace
+
+// =====================================================================  ABI
+extern "C" {
+
+const char* mxq_status_string(mxq_status s) {
+  switch (s) {
+    case MXQ_OK: return "ok";
+    case MXQ_ERR_INVALID_ARG: return "invalid argument";
+    case MXQ_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+    case MXQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MXQ_ERR_WORKSPACE: return "workspace or storage too small";
+    case MXQ_ERR_ARCH: return "no sm_100 CUDA device";
+    case MXQ_ERR_CUDA: return "CUDA error";
+    case MXQ_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+int mxq_version(void) { return (1 << 16) | 0; }
+
+int mxq_last_cuda_error(void) { return t_last_cuda_error; }
+
+size_t mxq_sf_bytes(int64_t rows, int64_t k, mxq_format f) {
+  if (rows < 0 || k < 0) return 0;
+  if (f == MXQ_NVFP4) return static_cast<size_t>(pad_to(rows, 128) * pad_to(k / 16, 4));
+  if (f == MXQ_MXFP8) return static_cast<size_t>(pad_to(rows, 128) * pad_to(k / 32, 4));
+  return 0;
+}
+
+size_t mxq_codes_bytes(int64_t rows, int64_t k, mxq_format f) {
+  if (rows < 0 || k < 0) return 0;
+  if (f == MXQ_NVFP4) return static_cast<size_t>(rows * k / 2);
+  if (f == MXQ_MXFP8) return static_cast<size_t>(rows * k);
+  if (f == MXQ_BF16) return static_cast<size_t>(rows * k * 2);
+  return 0;
+}
+
+mxq_status mxq_amax(const void* x_bf16, int64_t rows, int64_t k, int64_t ld, float* amax_dev,
+                    mxq_stream_t stream) {
+  if (amax_dev == nullptr) return MXQ_ERR_INVALID_ARG;
+  mxq_status st = check_bf16_matrix(x_bf16, rows, k, ld);
+  if (st != MXQ_OK) return st;
+  if (k % 8 != 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  if (reinterpret_cast<uintptr_t>(amax_dev) & 3u) return MXQ_ERR_ALIGNMENT;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+  return launch_amax(x_bf16, rows, k, ld, amax_dev, reinterpret_cast<cudaStream_t>(stream), sms);
+}
+
+mxq_status mxq_quantize_nvfp4(const void* x_bf16, int64_t rows, int64_t k, int64_t ld,
+                              const float* amax_dev, uint8_t* codes, uint8_t* sf_swz,
+                              float* g_dev, mxq_stream_t stream) {
+  mxq_status st = check_bf16_matrix(x_bf16, rows, k, ld);
+  if (st != MXQ_OK) return st;
+  if (amax_dev == nullptr || g_dev == nullptr) return MXQ_ERR_INVALID_ARG;
+  if (rows > 0 && k > 0 && (codes == nullptr || sf_swz == nullptr)) return MXQ_ERR_INVALID_ARG;
+  if (k % 64 != 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(codes) || !aligned16(sf_swz)) return MXQ_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(amax_dev) & 3u) || (reinterpret_cast<uintptr_t>(g_dev) & 3u))
+    return MXQ_ERR_ALIGNMENT;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+  if (rows == 0 || k == 0) return MXQ_OK;
+  return launch_quant_nvfp4(x_bf16, rows, k, ld, amax_dev, codes, sf_swz, g_dev,
+                            reinterpret_cast<cudaStream_t>(stream), sms);
+}
+
+mxq_status mxq_quantize_mxfp8(const void* x_bf16, int64_t rows, int64_t k, int64_t ld,
+                              uint8_t* codes, uint8_t* sf_swz, mxq_stream_t stream) {
+  mxq_status st = check_bf16_matrix(x_bf16, rows, k, ld);
+  if (st != MXQ_OK) return st;
+  if (rows > 0 && k > 0 && (codes == nullptr || sf_swz == nullptr)) return MXQ_ERR_INVALID_ARG;
+  if (k % 128 != 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(codes) || !aligned16(sf_swz)) return MXQ_ERR_ALIGNMENT;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+  if (rows == 0 || k == 0) return MXQ_OK;
+  return launch_quant_mxfp8(x_bf16, rows, k, ld, codes, sf_swz,
+                            reinterpret_cast<cudaStream_t>(stream), sms);
+}
+
+mxq_status mxq_gemm_blockscaled(mxq_format f, int64_t M, int64_t N, int64_t K,
+                                const void* a_codes, const uint8_t* a_sf, const float* a_g_dev,
+                                const void* b_codes, const uint8_t* b_sf, const float* b_g_dev,
+                                const void* bias_bf16, void* y_bf16, int64_t ldy,
+                                mxq_stream_t stream) {
+  if (!valid_format(f)) return MXQ_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0) return MXQ_ERR_INVALID_ARG;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  if (K == 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  if (f == MXQ_NVFP4 && K % 64 != 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  if (f == MXQ_MXFP8 && K % 128 != 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  if (f == MXQ_BF16 && K % 8 != 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  if (ldy < N || ldy < 1) return MXQ_ERR_INVALID_ARG;
+  if (ldy % 8 != 0) return MXQ_ERR_ALIGNMENT;
+  const bool nonempty = M > 0 && N > 0;
+  if (nonempty) {
+    if (a_codes == nullptr || b_codes == nullptr || y_bf16 == nullptr) return MXQ_ERR_INVALID_ARG;
+    if (f != MXQ_BF16 && (a_sf == nullptr || b_sf == nullptr)) return MXQ_ERR_INVALID_ARG;
+    if (f == MXQ_NVFP4 && (a_g_dev == nullptr || b_g_dev == nullptr)) return MXQ_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(y_bf16)) return MXQ_ERR_ALIGNMENT;
+    if (f != MXQ_BF16 && (!aligned16(a_sf) || !aligned16(b_sf))) return MXQ_ERR_ALIGNMENT;
+    if (bias_bf16 != nullptr && (reinterpret_cast<uintptr_t>(bias_bf16) & 1u)) return MXQ_ERR_ALIGNMENT;
+  }
+  int dev, sms;
+  mxq_status st;
+  if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+  if (!nonempty) return MXQ_OK;
+  if ((st = get_encoder()) != MXQ_OK) return st;
+  return launch_gemm(f, dev, sms, M, N, K, a_codes, a_sf, a_g_dev, b_codes, b_sf, b_g_dev,
+                     bias_bf16, y_bf16, ldy, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t mxq_weight_storage_bytes(int64_t N, int64_t K, mxq_format f) {
+  if (f != MXQ_NVFP4 && f != MXQ_MXFP8) return 0;
+  if (N < 0 || K < 0) return 0;
+  return quant_layout(N, K, f).total;
+}
+
+mxq_status mxq_weight_prepare(mxq_format f, const void* w_bf16, int64_t N, int64_t K,
+                              const void* bias_bf16, int keep_bf16, void* storage,
+                              size_t storage_bytes, mxq_weight* out, mxq_stream_t stream) {
+  if (out == nullptr || !valid_format(f)) return MXQ_ERR_INVALID_ARG;
+  mxq_status st = check_bf16_matrix(w_bf16, N, K, K);
+  if (st != MXQ_OK) return st;
+  if (bias_bf16 != nullptr && (reinterpret_cast<uintptr_t>(bias_bf16) & 1u)) return MXQ_ERR_ALIGNMENT;
+  mxq_weight w;
+  std::memset(&w, 0, sizeof(w));
+  w.format = f;
+  w.keep_bf16 = keep_bf16 ? 1 : 0;
+  w.N = N;
+  w.K = K;
+  w.w_bf16 = w_bf16;
+  w.bias_bf16 = bias_bf16;
+  const bool quantize = (f != MXQ_BF16) && !keep_bf16;
+  if (quantize) {
+    if (f == MXQ_NVFP4 && K % 64 != 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
+    if (f == MXQ_MXFP8 && K % 128 != 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
+    const QuantLayout l = quant_layout(N, K, f);
+    if (storage == nullptr) return MXQ_ERR_INVALID_ARG;
+    if (!aligned256(storage)) return MXQ_ERR_ALIGNMENT;
+    if (storage_bytes < l.total) return MXQ_ERR_WORKSPACE;
+    uint8_t* base = static_cast<uint8_t*>(storage);
+    float* amax = reinterpret_cast<float*>(base);
+    float* g = reinterpret_cast<float*>(base + 4);
+    uint8_t* codes = base + l.codes_off;
+    uint8_t* sf = base + l.sf_off;
+    int dev, sms;
+    if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (f == MXQ_NVFP4) {
+      if ((st = launch_amax(w_bf16, N, K, K, amax, s, sms)) != MXQ_OK) return st;
+      if (N > 0 && K > 0 &&
+          (st = launch_quant_nvfp4(w_bf16, N, K, K, amax, codes, sf, g, s, sms)) != MXQ_OK)
+        return st;
+      w.g_dev = g;
+      w.amax_dev = amax;
+    } else {
+      if (N > 0 && K > 0 && (st = launch_quant_mxfp8(w_bf16, N, K, K, codes, sf, s, sms)) != MXQ_OK)
+        return st;
+    }
+    w.codes = codes;
+    w.sf = sf;
+  }
+  *out = w;
+  return MXQ_OK;
+}
+
+int mxq_linear_path(const mxq_weight* w, int64_t M, const mxq_linear_opts* opts) {
+  if (w == nullptr) return 0;
+  const int64_t min_dim = (opts != nullptr && opts->min_dim > 0) ? opts->min_dim : 1024;
+  if (w->keep_bf16 || w->format == MXQ_BF16) return MXQ_BF16;
+  int64_t m = M < w->K ? M : w->K;
+  m = m < w->N ? m : w->N;
+  if (m < min_dim) return MXQ_BF16;
+  return w->format;
+}
+
+size_t mxq_linear_workspace_bytes(int64_t M, int64_t K, mxq_format f) {
+  if (f != MXQ_NVFP4 && f != MXQ_MXFP8) return 0;
+  if (M < 0 || K < 0) return 0;
+  return quant_layout(M, K, f).total;
+}
+
+mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* y_bf16, void* ws,
+                      size_t ws_bytes, const mxq_linear_opts* opts, mxq_stream_t stream) {
+  if (w == nullptr || !valid_format(w->format)) return MXQ_ERR_INVALID_ARG;
+  const int64_t N = w->N, K = w->K;
+  mxq_status st = check_bf16_matrix(x_bf16, M, K, K);
+  if (st != MXQ_OK) return st;
+  if (M > 0 && N > 0 && y_bf16 == nullptr) return MXQ_ERR_INVALID_ARG;
+  if (!aligned16(y_bf16)) return MXQ_ERR_ALIGNMENT;
+  if (N % 8 != 0) return MXQ_ERR_ALIGNMENT;  // y rows are N elements apart
+  const int path = mxq_linear_path(w, M, opts);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (path == MXQ_BF16) {
+    if (M > 0 && N > 0 && w->w_bf16 == nullptr) return MXQ_ERR_INVALID_ARG;
+    return mxq_gemm_blockscaled(MXQ_BF16, M, N, K, x_bf16, nullptr, nullptr, w->w_bf16, nullptr,
+                                nullptr, w->bias_bf16, y_bf16, N, stream);
+  }
+  const mxq_format f = static_cast<mxq_format>(path);
+  if (w->codes == nullptr || w->sf == nullptr) return MXQ_ERR_INVALID_ARG;
+  if (f == MXQ_NVFP4 && w->g_dev == nullptr) return MXQ_ERR_INVALID_ARG;
+  const QuantLayout l = quant_layout(M, K, f);
+  if (ws == nullptr) return MXQ_ERR_INVALID_ARG;
+  if (!aligned256(ws)) return MXQ_ERR_ALIGNMENT;
+  if (ws_bytes < l.total) return MXQ_ERR_WORKSPACE;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+  if (M == 0 || N == 0) return MXQ_OK;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* amax = reinterpret_cast<float*>(base);
+  float* g = reinterpret_cast<float*>(base + 4);
+  uint8_t* codes = base + l.codes_off;
+  uint8_t* sf = base + l.sf_off;
+  if (f == MXQ_NVFP4) {
+    if ((st = launch_amax(x_bf16, M, K, K, amax, s, sms)) != MXQ_OK) return st;
+    if ((st = launch_quant_nvfp4(x_bf16, M, K, K, amax, codes, sf, g, s, sms)) != MXQ_OK) return st;
+  } else {
+    if ((st = launch_quant_mxfp8(x_bf16, M, K, K, codes, sf, s, sms)) != MXQ_OK) return st;
+  }
+  if ((st = get_encoder()) != MXQ_OK) return st;
+  return launch_gemm(f, dev, sms, M, N, K, codes, sf, g, w->codes, w->sf, w->g_dev, w->bias_bf16,
+                     y_bf16, N, s);
+}
+
+mxq_status mxq_get_device_error(mxq_stream_t stream) {
+  int dev, sms;
+  mxq_status st = current_device(&dev, &sms);
+  if (st != MXQ_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, mxq::g_device_error, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (v != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(mxq::g_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return MXQ_ERR_TIMEOUT;
+  }
+  return MXQ_OK;
+}
+
+mxq_status mxq_convert_f32(const float* in, int64_t n, int code_fmt, uint8_t* out,
+                           mxq_stream_t stream) {
+  if (n < 0 || (code_fmt != 1 && code_fmt != 2)) return MXQ_ERR_INVALID_ARG;
+  if (n > 0 && (in == nullptr || out == nullptr)) return MXQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(in) & 3u) return MXQ_ERR_ALIGNMENT;
+  int dev, sms;
+  mxq_status st = current_device(&dev, &sms);
+  if (st != MXQ_OK) return st;
+  if (n == 0) return MXQ_OK;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
+  mxq::convert_kernel<<<static_cast<int>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      in, n, code_fmt, out);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -24,3 +24,17 @@ def pytest_collection_modifyitems(config, items):
     # A GPU test on a machine without a GPU is an error in the caller's
     # selection, not something to skip silently: fail loudly.
     pass
+
+
+def _ensure_library_built():
+    """Build libmxq.so in-tree when it is missing or older than its sources
+    (loads the build script by path: importing the package needs the library)."""
+    import importlib.util
+    path = os.path.join(ROOT, "fp8_gemm_diffusion_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_mxq_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+_ensure_library_built()

@@ -143,6 +143,14 @@ CONFIG_NAMES = {
 }
 
 
+CASE_NAMES = {
+    "c1": "c1_nvfp4_256x1024x1024",
+    "c2": "c2_mxfp8_4608x3072x9216",
+    "c3": "c3_nvfp4_4608x3072x12288",
+    "c4": "c4_nvfp4_16896x12288x3072",
+}
+
+
 def make_case(name: str, **kw) -> LinearCase:
     return CONFIG_NAMES[name](**kw)
 
