@@ -93,6 +93,8 @@ _linear_path = _proto("mxq_linear_path", _int, ctypes.POINTER(mxq_weight), _i64,
 _linear_workspace_bytes = _proto("mxq_linear_workspace_bytes", _sz, _i64, _i64, _int)
 _linear = _proto("mxq_linear", _int, ctypes.POINTER(mxq_weight), _ptr, _i64, _ptr, _ptr, _sz,
                  ctypes.POINTER(mxq_linear_opts), _ptr)
+_linear_noalloc = _proto("mxq_linear_noalloc", _int, ctypes.POINTER(mxq_weight), _ptr, _i64,
+                         _ptr, ctypes.POINTER(mxq_linear_opts), _ptr)
 _get_device_error = _proto("mxq_get_device_error", _int, _ptr)
 _convert_f32 = _proto("mxq_convert_f32", _int, _ptr, _i64, _int, _ptr, _ptr)
 
@@ -102,8 +104,11 @@ EXPORTED = [
     "mxq_codes_bytes", "mxq_amax", "mxq_quantize_nvfp4", "mxq_quantize_mxfp8",
     "mxq_gemm_blockscaled", "mxq_weight_storage_bytes", "mxq_weight_prepare",
     "mxq_linear_path", "mxq_linear_workspace_bytes", "mxq_linear", "mxq_get_device_error",
-    "mxq_convert_f32",
+    "mxq_convert_f32", "mxq_linear_noalloc",
 ]
+
+#: Capacity of the static device scratch of mxq_linear_noalloc (MXQ_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 class MxqError(RuntimeError):
@@ -229,6 +234,15 @@ def linear_workspace_bytes(M: int, K: int, fmt) -> int:
 def linear(w: mxq_weight, x, M, y, ws, ws_bytes, min_dim=None, stream=None) -> None:
     _check(_linear(ctypes.byref(w), _addr(x), M, _addr(y), _addr(ws), ws_bytes, _opts(min_dim),
                    _stream(stream)), "mxq_linear")
+
+
+def linear_noalloc(w: mxq_weight, x, M, y, min_dim=None, stream=None) -> None:
+    """mxq_linear without a workspace argument, for callers that cannot
+    allocate device memory (fixed memory budget, or no cudaMalloc allowed in a
+    latency-critical loop): the library's static device scratch is used
+    instead.  Calls that overlap on the GPU race on that shared scratch."""
+    _check(_linear_noalloc(ctypes.byref(w), _addr(x), M, _addr(y), _opts(min_dim),
+                           _stream(stream)), "mxq_linear_noalloc")
 
 
 def get_device_error(stream=None) -> int:

@@ -219,6 +219,34 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
                       void* ws, size_t ws_bytes, const mxq_linear_opts* opts,
                       mxq_stream_t stream);
 
+/* Size of the device scratch array that mxq_linear_noalloc uses (64 MiB). */
+#define MXQ_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * mxq_linear_noalloc - mxq_linear for callers that cannot allocate device
+ * memory: for example a host whose device-memory budget is fixed at start-up
+ * and that forbids allocations afterwards, or a latency-critical loop where
+ * cudaMalloc (it may synchronise the device and its latency is unbounded) is
+ * not acceptable.  The paper has no counterpart: it is an addition of this
+ * library.
+ * Same arguments and result as mxq_linear, without ws / ws_bytes: the
+ * workspace for the quantised activation lives in a file-scope device array of
+ * MXQ_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until
+ * the process exits.  Nothing is allocated by the call.
+ *  - The first call on a device (with that device current) looks up the
+ *    array's address and caches it; make that first call before any stream
+ *    capture.
+ *  - All calls share the array and it keeps the previous call's contents; the
+ *    one value that must start at zero (the activation amax) is cleared on the
+ *    stream by every call.  Calls that can overlap on the GPU (other streams,
+ *    unordered host threads) race on the array: serialise them.
+ *  - A quantised path whose workspace (mxq_linear_workspace_bytes) exceeds
+ *    MXQ_NOALLOC_SCRATCH_BYTES returns MXQ_ERR_WORKSPACE and enqueues nothing;
+ *    the bf16 path needs no workspace.
+ */
+mxq_status mxq_linear_noalloc(const mxq_weight* w, const void* x_bf16, int64_t M, void* y_bf16,
+                              const mxq_linear_opts* opts, mxq_stream_t stream);
+
 /* ---------------------------------------------------- diagnostics ------- */
 
 /*
