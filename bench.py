@@ -126,6 +126,22 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples)}
 
 
+# ------------------------------------------------------- rank aggregation
+def max_over_ranks(ms: float, device) -> float:
+    """Max of a per-rank time over all ranks (identity without a process group)."""
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, steps: int, flops_per_step: float, max_ms: float) -> float:
+    """Whole-job throughput: every replica did `steps` steps in at most max_ms."""
+    return world * steps * flops_per_step / (max_ms * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------ the GPU arm
 def run_gpu(args, rank, world, local_rank):
     import fp8_gemm_diffusion_b200 as mxq
@@ -224,10 +240,7 @@ def run_gpu(args, rank, world, local_rank):
     gemm_ms = [e[2].elapsed_time(e[3]) for e in evs]
     if mxq.get_device_error() != mxq.OK:
         raise RuntimeError("device-side timeout during the timed steps")
-    if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
 
     # end to end through the public call with host buffers
     e2e = run_e2e(mxq, case, base_w, dev, stream, args, dist)
@@ -236,7 +249,7 @@ def run_gpu(args, rank, world, local_rank):
     peak = peaks["bf16"] * NOMINAL_RATIO[fmt]
     gemm_avg_s = float(np.mean(gemm_ms)) * 1e-3
     achieved = flops / gemm_avg_s / 1e12
-    value = world * args.steps * flops / (total_ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, args.steps, flops, total_ms)
     qbytes = (M * K * 2 + M * K // (2 if fmt == "nvfp4" else 1)
               + mxq.sf_bytes(M, K, fmt))
     result = {
@@ -317,14 +330,10 @@ def run_e2e(mxq, case, base_w, dev, stream, args, dist):
         one()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(a.elapsed_time(b), dev)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     flops = 2.0 * M * N * K
-    return {"value": round(world * steps * flops / (ms * 1e-3) / 1e12, 3), "unit": UNIT,
+    return {"value": round(whole_job_tflops(world, steps, flops, ms), 3), "unit": UNIT,
             "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "steps": steps}
 
 
