@@ -1,0 +1,462 @@
+// gemm_pair.cuh - block-scaled GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+// Same result as gemm.cuh, Y = bf16(alpha * A.B^T + bias), computed with
+// 256 x BN output tiles on a pair of CTAs in one cluster (the "CTA pair" of
+// the WaveSpeedAI x DataCrunch B200 article, section "NVIDIA's Blackwell GPU
+// architecture: B200"): each CTA loads its own 128 rows of A and BN/2 rows of
+// B, and the even CTA of the pair issues M=256 MMAs that read A and B from
+// both CTAs' shared memory and leave each CTA's 128 rows of D in that CTA's
+// tensor memory.  Per CTA this halves the operand traffic of a 128 x BN tile
+// and the pair MMA runs the tensor cores at a higher rate than M=128 MMAs.
+//
+// Roles (both CTAs):
+//   warp 0      A/B producer: each stage's 128 rows of A and BN/2 rows of B
+//               into this CTA's ring; completions land on the even CTA's full
+//               barrier (cta_group::2 loads, no multicast).
+//   warp 1      tensor memory (cta_group::2 allocation); on the even CTA one
+//               lane issues the MMAs and commits to both CTAs' barriers
+//               (multicast commit): A/B stage free, scale set free, and
+//               accumulator full.
+//   warp 2      scale loader: the scale chunks of each stage (A's 128 rows and
+//               all BN columns of B: each CTA's tensor memory needs B's) into
+//               a separate ring that runs ahead of the A/B ring.
+//   warps 3-6   scale writers, one per tensor-memory sub-partition: chunk rows
+//               from shared memory into a per-stage set of tensor-memory
+//               columns with tcgen05.st, so no tcgen05.cp sits between MMAs.
+//               They run up to NS stages ahead of the MMAs.
+//   warps 7-10  epilogue, one per sub-partition: 128 accumulator columns per
+//               batch into registers, release the accumulator after the last
+//               batch, then alpha, bias, bf16, 128-byte swizzled staging and
+//               TMA stores.
+// Every wait is bounded (ptx.cuh); a timed-out role stops, loads and MMAs in
+// flight are drained, and both CTAs free tensor memory together.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <cstdint>
+
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace mxq {
+
+template <Fmt F, int BN_>
+struct PairCfg {
+  static constexpr int BM = 256;      // rows of a pair tile
+  static constexpr int BM_CTA = 128;  // rows per CTA
+  static constexpr int BN = BN_;
+  static constexpr int BN_CTA = BN / 2;
+  static_assert(BN == 128 || BN == 256, "BN: the epilogue drains 128-column batches");
+  static constexpr int ROW_BYTES = 128;
+  static constexpr int K_STAGE = F == Fmt::NVFP4 ? 256 : (F == Fmt::MXFP8 ? 128 : 64);
+  static constexpr int MMA_K = F == Fmt::NVFP4 ? 64 : (F == Fmt::MXFP8 ? 32 : 16);
+  static constexpr int MMAS = K_STAGE / MMA_K;
+  static constexpr bool SCALED = F != Fmt::BF16;
+  static constexpr int NRB = (BN + 127) / 128;  // 128-row scale blocks of the pair's B tile
+  static constexpr int SF_CHUNKS = F == Fmt::NVFP4 ? MMAS : (F == Fmt::MXFP8 ? 1 : 0);  // per 128 rows
+  static constexpr int SF_BOX_ROWS = SF_CHUNKS * 2;  // scales are loaded as [rows][256 B]
+  static constexpr int A_BYTES = BM_CTA * ROW_BYTES;
+  static constexpr int B_BYTES = BN_CTA * ROW_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // multiple of 1024
+  static constexpr uint32_t AB_PAIR_TX = 2u * STAGE_BYTES;  // A/B of both CTAs
+  static constexpr int SFA_BYTES = SF_CHUNKS * 512;
+  static constexpr int SFB_BYTES = NRB * SF_CHUNKS * 512;
+  static constexpr uint32_t SF_TX = SFA_BYTES + SFB_BYTES;  // this CTA's scales
+  static constexpr int SF_SLOT_BYTES = SCALED ? (SFA_BYTES + SFB_BYTES + 1023) / 1024 * 1024 : 0;
+  static constexpr int SF_SLOTS = SCALED ? (F == Fmt::NVFP4 ? 4 : 8) : 0;
+  // tensor memory: the accumulator (BN columns), then NS scale sets (A chunks,
+  // then B chunks in MMA-major order, 4 columns each)
+  static constexpr int SF_SET_COLS = (SF_CHUNKS + NRB * SF_CHUNKS) * 4;
+  static constexpr int SF_COL = BN;
+  static constexpr int SFB_OFF = SF_CHUNKS * 4;
+  static constexpr int TMEM_COLS = 512;
+  // one scale set per A/B stage: a set is free when its stage is (same commit)
+  static constexpr int NS_FIT = SCALED ? (TMEM_COLS - BN) / SF_SET_COLS : 64;
+  static constexpr int SF_WARPS = 4;   // one per tensor-memory sub-partition
+  static constexpr int EPI_WARPS = 4;  // one per sub-partition
+  static constexpr int EPI_BATCHES = BN / 128;
+  static constexpr int EPI_BYTES = EPI_WARPS * 32 * 128 * 2;  // one 128-column batch per warp
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int STAGES_FIT =
+      (232448 - 1024 - BAR_BYTES - EPI_BYTES - SF_SLOTS * SF_SLOT_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_MIN = STAGES_FIT < NS_FIT ? STAGES_FIT : NS_FIT;
+  static constexpr int STAGES = STAGES_MIN > 6 ? 6 : STAGES_MIN;
+  static constexpr int NS = STAGES;
+  static_assert(STAGES >= 2, "shared / tensor memory");
+  static constexpr int SMEM_BYTES =
+      1024 + STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + EPI_BYTES + BAR_BYTES;
+  static constexpr int THREADS = 32 * (3 + SF_WARPS + EPI_WARPS);
+};
+
+// Instruction descriptor of an M=256 (pair) MMA; fields as in make_idesc.
+template <Fmt F>
+__device__ __forceinline__ uint32_t make_idesc_pair(int n, uint32_t sf_id) {
+  const uint32_t m_field = (256u >> 4) << 24;
+  const uint32_t n_field = (static_cast<uint32_t>(n) >> 3) << 17;
+  if constexpr (F == Fmt::NVFP4) {
+    return (sf_id << 4) | (1u << 7) | (1u << 10) | n_field | m_field | (sf_id << 29);
+  } else if constexpr (F == Fmt::MXFP8) {
+    return (sf_id << 4) | n_field | (1u << 23) | m_field | (sf_id << 29);
+  } else {
+    return (1u << 4) | (1u << 7) | (1u << 10) | n_field | m_field;
+  }
+}
+
+struct PairArgs {
+  int M, N, K;
+  const float* a_g;
+  const float* b_g;
+  const __nv_bfloat16* bias;
+};
+
+template <Fmt F, int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                     const __grid_constant__ CUtensorMap tmap_b,
+                     const __grid_constant__ CUtensorMap tmap_sfa,
+                     const __grid_constant__ CUtensorMap tmap_sfb,
+                     const __grid_constant__ CUtensorMap tmap_y, const PairArgs args) {
+  using C = PairCfg<F, BN>;
+  constexpr int S = C::STAGES, R = C::SF_SLOTS, NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw_addr);
+  const uint32_t sf_base = base + S * C::STAGE_BYTES;
+  const uint32_t epi_base = sf_base + R * C::SF_SLOT_BYTES;
+  const uint32_t bar_base = epi_base + C::EPI_BYTES;
+  // barriers: [full S][empty S][sf_full R][sf_empty R][sf_ready S][tfull][tempty][drain]
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };                 // even CTA: A/B landed
+  auto empty_bar = [&](int s) { return bar_base + 8u * (S + s); };          // both: A/B stage free
+  auto sf_full_bar = [&](int r) { return bar_base + 8u * (2 * S + r); };    // both: own scales landed
+  auto sf_empty_bar = [&](int r) { return bar_base + 8u * (2 * S + R + r); };  // both: slot read
+  auto sf_ready_bar = [&](int n) { return bar_base + 8u * (2 * S + 2 * R + n); };  // even: set written
+  const uint32_t tfull_bar = bar_base + 8u * (2 * S + 2 * R + NS);
+  const uint32_t tempty_bar = tfull_bar + 8u;
+  const uint32_t drain_bar = tfull_bar + 16u;
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + (tfull_bar + 24u - base));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs of the pair
+
+  const int M = args.M, N = args.N, K = args.K;
+  const int m_tiles = (M + C::BM - 1) / C::BM;
+  const int n_tiles = (N + BN - 1) / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int num_kb = (K + C::K_STAGE - 1) / C::K_STAGE;
+  const int sf_c4 = F == Fmt::NVFP4 ? K / 64 : (F == Fmt::MXFP8 ? K / 128 : 0);
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+  const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / num_pairs + 1 : 0;
+  const int total_kb = my_tiles * num_kb;  // stages this pair runs
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int r = 0; r < R; ++r) {
+      mbar_init(sf_full_bar(r), 1);
+      mbar_init(sf_empty_bar(r), C::SF_WARPS);
+    }
+    for (int n = 0; n < NS; ++n) mbar_init(sf_ready_bar(n), 2 * C::SF_WARPS);
+    mbar_init(tfull_bar, 1);
+    mbar_init(tempty_bar, 2 * C::EPI_WARPS);
+    mbar_init(drain_bar, 1);
+    fence_barrier_init();
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    prefetch_tmap(&tmap_y);
+    if constexpr (C::SCALED) {
+      prefetch_tmap(&tmap_sfa);
+      prefetch_tmap(&tmap_sfb);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ A/B producer
+    if (lane == 0) {
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      const int a_row_off = static_cast<int>(rank) * C::BM_CTA;
+      const int b_row_off = static_cast<int>(rank) * C::BN_CTA;
+      constexpr int KX = C::ROW_BYTES / (F == Fmt::BF16 ? 2 : 1);  // K coordinate step per stage
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        const int nt = tile / m_tiles, mt = tile - nt * m_tiles;
+        const int a_row = mt * C::BM + a_row_off, b_row = nt * BN + b_row_off;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(s), C::AB_PAIR_TX);
+          const uint32_t leader_full = map_to_cta(full_bar(s), 0);
+          const uint32_t sa = base + s * C::STAGE_BYTES;
+          tma_load_2d_pair(sa, &tmap_a, leader_full, kb * KX, a_row);
+          tma_load_2d_pair(sa + C::A_BYTES, &tmap_b, leader_full, kb * KX, b_row);
+          ++issued;
+          if (++s == S) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok && rank == 0) {
+        // let every armed stage land before the pair can exit
+        for (int i = 0; i < S && i < issued; ++i) {
+          if (--s < 0) { s = S - 1; ph ^= 1u; }
+          mbar_wait_bounded(full_bar(s), ph);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // (one thread: keep the per-stage work to a few instructions)
+    if (lane == 0 && rank == 0) {
+      int s = 0;
+      uint32_t ph = 0, acc_ph = 0;
+      bool ok = true;
+      const uint64_t adesc0 = desc_kmajor_sw128(base);
+      const uint64_t bdesc0 = desc_kmajor_sw128(base + C::A_BYTES);
+      constexpr uint64_t DSTEP = C::STAGE_BYTES >> 4;  // descriptor start-address step per stage
+      const uint32_t idesc = make_idesc_pair<F>(BN, 0);
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        const int nt = tile / m_tiles;
+        const uint32_t sfb_shift = ((nt * BN) & 127) >> 5;
+        // the accumulator is single-buffered: wait until the epilogue has read the last tile
+        if (!mbar_wait_bounded(tempty_bar, acc_ph ^ 1u)) { ok = false; break; }
+        acc_ph ^= 1u;
+        tc_fence_after();
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(full_bar(s), ph)) { ok = false; break; }
+          if (C::SCALED && !mbar_wait_bounded(sf_ready_bar(s), ph)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = adesc0 + DSTEP * s, bdesc = bdesc0 + DSTEP * s;
+          const uint32_t sf = tmem_base + C::SF_COL + s * C::SF_SET_COLS;
+          int nmma = C::MMAS;
+          if constexpr (F == Fmt::NVFP4) {
+            if (kb == num_kb - 1) nmma = K / 64 - kb * C::MMAS;  // K % 256 != 0: partial last stage
+          }
+#pragma unroll
+          for (int j = 0; j < C::MMAS; ++j) {
+            if (j < nmma) {
+              const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
+              const uint64_t koff = static_cast<uint64_t>(2 * j);  // 32 bytes of K per MMA
+              if constexpr (F == Fmt::NVFP4) {
+                mma_pair_nvfp4(tmem_base, adesc + koff, bdesc + koff, idesc, sf + 4 * j,
+                               sf + C::SFB_OFF + j * C::NRB * 4 + sfb_shift, accum);
+              } else if constexpr (F == Fmt::MXFP8) {
+                const uint32_t id = static_cast<uint32_t>(j) << 30;
+                mma_pair_mxfp8(tmem_base, adesc + koff, bdesc + koff,
+                               idesc | (static_cast<uint32_t>(j) << 4) | (static_cast<uint32_t>(j) << 29),
+                               sf | id, (sf + C::SFB_OFF + sfb_shift) | id, accum);
+              } else {
+                mma_pair_bf16(tmem_base, adesc + koff, bdesc + koff, idesc, accum);
+              }
+            }
+          }
+          tc_commit_pair(empty_bar(s));  // frees A/B stage s and scale set s
+          if (++s == S) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair(tfull_bar);
+      }
+      tc_commit_pair(drain_bar);
+      mbar_wait_bounded(drain_bar, 0);
+    } else if (lane == 0) {
+      // odd CTA: the pair's MMAs read this CTA's memory; wait for the last one
+      mbar_wait_bounded(drain_bar, 0);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale loader
+    if constexpr (C::SCALED) if (lane == 0) {
+      int r = 0, issued = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        const int nt = tile / m_tiles, mt = tile - nt * m_tiles;
+        // 512-byte chunk (row block rb, 4-column group kc) is 256-byte row 2*(rb*sf_c4+kc)
+        const int ya = 2 * (mt * 2 + static_cast<int>(rank)) * sf_c4;
+        const int yb = 2 * (nt * BN / 128) * sf_c4;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(sf_empty_bar(r), ph ^ 1u)) { ok = false; break; }
+          mbar_arrive_expect_tx(sf_full_bar(r), C::SF_TX);
+          const uint32_t slot = sf_base + r * C::SF_SLOT_BYTES;
+          const int kc2 = 2 * kb * C::SF_CHUNKS;
+          tma_load_2d(slot, &tmap_sfa, sf_full_bar(r), 0, ya + kc2);
+#pragma unroll
+          for (int c = 0; c < C::NRB; ++c)
+            tma_load_2d(slot + C::SFA_BYTES + c * C::SFA_BYTES, &tmap_sfb, sf_full_bar(r), 0,
+                        yb + 2 * c * sf_c4 + kc2);
+          ++issued;
+          if (++r == R) { r = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) {
+        for (int i = 0; i < R && i < issued; ++i) {
+          if (--r < 0) { r = R - 1; ph ^= 1u; }
+          mbar_wait_bounded(sf_full_bar(r), ph);
+        }
+      }
+    }
+  } else if (warp < 3 + C::SF_WARPS) {
+    // ------------------------------------------------ scale factors -> TMEM
+    // Each warp writes the 32 lanes of its sub-partition: lane l receives row l
+    // of every 512-byte scale chunk of the stage (16 bytes = 4 columns), the
+    // layout the block-scaled MMA reads (row r's scales in lane r % 32 of
+    // every sub-partition, column r / 32 of the chunk's four).
+    if constexpr (C::SCALED) {
+      const uint32_t q = static_cast<uint32_t>(warp & 3);
+      const uint32_t leader_ready0 = map_to_cta(sf_ready_bar(0), 0);
+      constexpr int NCH = C::SF_CHUNKS * (1 + C::NRB);  // A chunks, then B chunks
+      int r = 0, n = 0;
+      uint32_t rph = 0, nph = 0;
+      for (int g = 0; g < total_kb; ++g) {
+        if (!mbar_wait_bounded(sf_full_bar(r), rph)) break;
+        const uint32_t slot = sf_base + r * C::SF_SLOT_BYTES;
+        uint32_t v[NCH * 4];
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          // TMEM order: A j, then B (j, c) MMA-major; the slot holds B as (c, j)
+          int off;
+          if (i < C::SF_CHUNKS) {
+            off = i * 512;
+          } else {
+            const int jb = (i - C::SF_CHUNKS) / C::NRB, cb = (i - C::SF_CHUNKS) % C::NRB;
+            off = C::SFA_BYTES + (cb * C::SF_CHUNKS + jb) * 512;
+          }
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v[4 * i]), "=r"(v[4 * i + 1]), "=r"(v[4 * i + 2]), "=r"(v[4 * i + 3])
+                       : "r"(slot + off + lane * 16));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sf_empty_bar(r));  // slot read: the loader may refill it
+        // the set is free once the MMAs of stage g - NS have completed
+        if (g >= NS && !mbar_wait_bounded(empty_bar(n), nph ^ 1u)) break;
+        tc_fence_after();
+        const uint32_t t = tmem_base + (q * 32u << 16) + C::SF_COL + n * C::SF_SET_COLS;
+        if constexpr (NCH * 4 % 16 == 0) {
+#pragma unroll
+          for (int i = 0; i < NCH * 4 / 16; ++i) {
+            uint32_t w[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) w[k] = v[16 * i + k];
+            tmem_st_32x32b_x16(t + 16 * i, w);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < NCH; ++i)
+            tmem_st_32x32b_x4(t + 4 * i, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(leader_ready0 + 8u * n);
+        if (++r == R) { r = 0; rph ^= 1u; }
+        if (++n == NS) { n = 0; nph ^= 1u; }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // tensor-memory sub-partition = 32-row slice
+    const uint32_t stage_buf = epi_base + (warp - 3 - C::SF_WARPS) * (32 * 128 * 2);
+    const uint32_t leader_tempty = map_to_cta(tempty_bar, 0);
+    float alpha = 1.0f;
+    if constexpr (F == Fmt::NVFP4) alpha = (*args.a_g) * (*args.b_g);
+    const bool bias_vec = args.bias != nullptr && (reinterpret_cast<uintptr_t>(args.bias) & 15u) == 0;
+    for (int i_tile = 0; i_tile < my_tiles; ++i_tile) {
+      const int tile = pair + i_tile * num_pairs;
+      const int mt = tile % m_tiles, nt = tile / m_tiles;
+      const int row0 = mt * C::BM + static_cast<int>(rank) * C::BM_CTA + q * 32;
+      // the tile's bias, prefetched before the accumulator is ready: lane l holds
+      // columns [8l, 8l + 8) of the tile as four packed bf16 pairs
+      uint32_t bias_l[4] = {0u, 0u, 0u, 0u};
+      if (args.bias != nullptr && lane * 8 < BN) {
+        const int c0 = nt * BN + lane * 8;
+        if (bias_vec && c0 + 8 <= N) {
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(args.bias + c0));
+          bias_l[0] = u.x; bias_l[1] = u.y; bias_l[2] = u.z; bias_l[3] = u.w;
+        } else {
+          const uint16_t* bs = reinterpret_cast<const uint16_t*>(args.bias);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t lo = (c0 + 2 * e < N) ? bs[c0 + 2 * e] : 0u;
+            const uint32_t hi = (c0 + 2 * e + 1 < N) ? bs[c0 + 2 * e + 1] : 0u;
+            bias_l[e] = lo | (hi << 16);
+          }
+        }
+      }
+      if (!mbar_wait_bounded(tfull_bar, i_tile & 1)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int bt = 0; bt < C::EPI_BATCHES; ++bt) {
+        // 128 accumulator columns at once; the last batch releases the accumulator
+        uint32_t r[128];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x32_nowait(t_row + bt * 128 + g * 32, r + 32 * g);
+        tc_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) reg_fence32(r + 32 * g);
+        if (bt == C::EPI_BATCHES - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(leader_tempty);  // accumulator may be overwritten
+        }
+        if (lane == 0) bulk_wait_group_read<0>();  // previous batch's stores have read the staging
+        __syncwarp();
+        const int col_base = nt * BN + bt * 128;
+        // 16 groups of 8 columns: bias (8 bf16), alpha * acc + bias, bf16, one 16-byte store
+        // into the staging (two sub-tiles of 32 rows x 64 columns, 128-byte swizzle)
+#pragma unroll
+        for (int j16 = 0; j16 < 16; ++j16) {
+          uint32_t bw[4];  // bias of columns [8 * (16 bt + j16), +8) from the lane holding them
+#pragma unroll
+          for (int e = 0; e < 4; ++e) bw[e] = __shfl_sync(0xffffffffu, bias_l[e], bt * 16 + j16);
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float v0 = __uint_as_float(r[8 * j16 + 2 * e]), v1 = __uint_as_float(r[8 * j16 + 2 * e + 1]);
+            if constexpr (F == Fmt::NVFP4) { v0 *= alpha; v1 *= alpha; }
+            v0 += __uint_as_float(bw[e] << 16);
+            v1 += __uint_as_float(bw[e] & 0xFFFF0000u);
+            const __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
+          const int j = j16 & 7;  // 16-byte chunk within the 128-byte row
+          const uint32_t addr = stage_buf + (j16 >> 3) * 4096 + lane * 128 + ((j ^ (lane & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]),
+                       "r"(pk[2]), "r"(pk[3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < M) {
+          for (int k = 0; k < 2; ++k) {
+            const int x = col_base + 64 * k;
+            if (x < N) tma_store_2d(&tmap_y, stage_buf + k * 4096, x, row0);
+          }
+          bulk_commit_group();
+        }
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace mxq

@@ -14,6 +14,7 @@
 
 #include "../../include/mxq.h"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -210,10 +211,93 @@ mxq_status launch_gemm_bn(int dev, int sms, int slot, int64_t M, int64_t N, int6
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
+template <mxq::Fmt F, int BN>
+mxq_status launch_gemm_pair(int dev, int sms, int slot, int64_t M, int64_t N, int64_t K,
+                            const void* a, const uint8_t* a_sf, const float* a_g, const void* b,
+                            const uint8_t* b_sf, const float* b_g, const void* bias, void* y,
+                            int64_t ldy, cudaStream_t s) {
+  using C = mxq::PairCfg<F, BN>;
+  auto kern = mxq::gemm_pair_kernel<F, BN>;
+  const uint32_t bit = 1u << slot;
+  if (!(g_dev[dev].smem_attr_set.load(std::memory_order_acquire) & bit)) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_dev[dev].smem_attr_set.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  CUtensorMap ta, tb, tsa, tsb, ty;
+  mxq_status st;
+  if (F == mxq::Fmt::BF16) {
+    st = tmap_2d(&ta, a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, K * 2, 64, C::BM_CTA,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st == MXQ_OK)
+      st = tmap_2d(&tb, b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, N, K * 2, 64, C::BN_CTA,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    tsa = ta;
+    tsb = tb;
+  } else {
+    const int64_t row_bytes = F == mxq::Fmt::NVFP4 ? K / 2 : K;
+    const mxq_format f = F == mxq::Fmt::NVFP4 ? MXQ_NVFP4 : MXQ_MXFP8;
+    st = tmap_2d(&ta, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, row_bytes, M, row_bytes, 128, C::BM_CTA,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st == MXQ_OK)
+      st = tmap_2d(&tb, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, row_bytes, N, row_bytes, 128, C::BN_CTA,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    // scale arrays viewed as rows of 256 bytes (a 512-byte chunk is two rows)
+    if (st == MXQ_OK)
+      st = tmap_2d(&tsa, a_sf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 256, mxq_sf_bytes(M, K, f) / 256, 256,
+                   256, C::SF_BOX_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st == MXQ_OK)
+      st = tmap_2d(&tsb, b_sf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 256, mxq_sf_bytes(N, K, f) / 256, 256,
+                   256, C::SF_BOX_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
+  if (st == MXQ_OK)
+    st = tmap_2d(&ty, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, ldy * 2, 64, 32,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != MXQ_OK) return st;
+  mxq::PairArgs args;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.a_g = a_g;
+  args.b_g = b_g;
+  args.bias = static_cast<const __nv_bfloat16*>(bias);
+  const int64_t tiles = ((M + C::BM - 1) / C::BM) * ((N + BN - 1) / BN);
+  const int64_t pairs = sms / 2;
+  const int grid = 2 * static_cast<int>(tiles < pairs ? tiles : pairs);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, tsa, tsb, ty, args);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
+}
+
 mxq_status launch_gemm(mxq_format f, int dev, int sms, int64_t M, int64_t N, int64_t K,
                        const void* a, const uint8_t* a_sf, const float* a_g, const void* b,
                        const uint8_t* b_sf, const float* b_g, const void* bias, void* y,
                        int64_t ldy, cudaStream_t s) {
+  if (M > 128) {
+    // CTA-pair kernel (M = 256 MMAs)
+    switch (f) {
+      case MXQ_NVFP4:
+        if (N > 128)
+          return launch_gemm_pair<mxq::Fmt::NVFP4, 256>(dev, sms, 6, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                        b_g, bias, y, ldy, s);
+        return launch_gemm_pair<mxq::Fmt::NVFP4, 128>(dev, sms, 7, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                      b_g, bias, y, ldy, s);
+      case MXQ_MXFP8:
+        if (N > 128)
+          return launch_gemm_pair<mxq::Fmt::MXFP8, 256>(dev, sms, 8, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                        b_g, bias, y, ldy, s);
+        return launch_gemm_pair<mxq::Fmt::MXFP8, 128>(dev, sms, 9, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                      b_g, bias, y, ldy, s);
+      case MXQ_BF16:
+        if (N > 128)
+          return launch_gemm_pair<mxq::Fmt::BF16, 256>(dev, sms, 10, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                       b_g, bias, y, ldy, s);
+        return launch_gemm_pair<mxq::Fmt::BF16, 128>(dev, sms, 11, M, N, K, a, a_sf, a_g, b, b_sf,
+                                                     b_g, bias, y, ldy, s);
+    }
+    return MXQ_ERR_INVALID_ARG;
+  }
   switch (f) {
     case MXQ_NVFP4:
       if (N % 192 == 0)

@@ -25,6 +25,11 @@ SHAPES = [
     (1, 64, 136),
     (333, 1024, 520),
     (640, 768, 1152),
+    # CTA-pair kernel edges: just above one CTA, a pair whose second CTA is
+    # entirely out of range, a 128-wide pair tile, ragged N on a 256-wide tile
+    (129, 256, 384),
+    (300, 512, 128),
+    (520, 1024, 136),
 ]
 
 
