@@ -110,10 +110,13 @@ mxq_status tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uin
   return MXQ_OK;
 }
 
-int quant_grid(int64_t vectors, int sms) {
-  const int64_t per_block = static_cast<int64_t>(mxq::kQuantThreads) * mxq::kQuantUnroll;
-  int64_t g = (vectors + per_block - 1) / per_block;
-  const int64_t cap = static_cast<int64_t>(sms) * 8;
+// One warp per row: enough blocks to give every row a warp, at most 8 blocks
+// per SM and at most kMaxAmaxPartials blocks (the partial-amax array size).
+int quant_grid(int64_t rows, int sms) {
+  const int64_t warps_per_block = mxq::kQuantThreads / 32;
+  int64_t g = (rows + warps_per_block - 1) / warps_per_block;
+  int64_t cap = static_cast<int64_t>(sms) * 8;
+  if (cap > mxq::kMaxAmaxPartials) cap = mxq::kMaxAmaxPartials;
   if (g > cap) g = cap;
   if (g < 1) g = 1;
   return static_cast<int>(g);
@@ -130,33 +133,46 @@ mxq_status check_bf16_matrix(const void* x, int64_t rows, int64_t k, int64_t ld)
 }
 
 // ----------------------------------------------------------------- launches
+// amax into one fp32 (zeroed first, then atomicMax of every block's maximum).
 mxq_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ld, float* amax,
                        cudaStream_t s, int sms) {
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
   if (e != cudaSuccess) return cuda_fail(e);
   if (rows == 0 || k == 0) return MXQ_OK;
-  const int64_t vectors = rows * (k / 8);
-  mxq::amax_kernel<<<quant_grid(vectors, sms), mxq::kQuantThreads, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(x), rows, k, ld, amax);
+  mxq::amax_kernel<<<quant_grid(rows, sms), mxq::kQuantThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<int>(rows), static_cast<int>(k), ld, nullptr,
+      amax);
   e = cudaGetLastError();
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
+// amax as per-block partial maxima (no zeroing needed); returns their count.
+mxq_status launch_amax_partials(const void* x, int64_t rows, int64_t k, int64_t ld, float* partials,
+                                int* n_partials, cudaStream_t s, int sms) {
+  const int grid = quant_grid(rows, sms);
+  mxq::amax_kernel<<<grid, mxq::kQuantThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
+                                                       static_cast<int>(rows), static_cast<int>(k),
+                                                       ld, partials, nullptr);
+  *n_partials = grid;
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
+}
+
 mxq_status launch_quant_nvfp4(const void* x, int64_t rows, int64_t k, int64_t ld,
-                              const float* amax, uint8_t* codes, uint8_t* sf, float* g,
-                              cudaStream_t s, int sms) {
-  const int64_t vectors = rows * (k / 8);
-  mxq::quantize_nvfp4_kernel<<<quant_grid(vectors, sms), mxq::kQuantThreads, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(x), rows, k, ld, amax, codes, sf, g);
+                              const float* amax_vals, int n_amax, uint8_t* codes, uint8_t* sf,
+                              float* g, float* amax_out, cudaStream_t s, int sms) {
+  mxq::quantize_nvfp4_kernel<<<quant_grid(rows, sms), mxq::kQuantThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<int>(rows), static_cast<int>(k), ld,
+      amax_vals, n_amax, codes, sf, g, amax_out);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
 mxq_status launch_quant_mxfp8(const void* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
                               uint8_t* sf, cudaStream_t s, int sms) {
-  const int64_t vectors = rows * (k / 8);
-  mxq::quantize_mxfp8_kernel<<<quant_grid(vectors, sms), mxq::kQuantThreads, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(x), rows, k, ld, codes, sf);
+  mxq::quantize_mxfp8_kernel<<<quant_grid(rows, sms), mxq::kQuantThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<int>(rows), static_cast<int>(k), ld, codes,
+      sf);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
@@ -323,14 +339,18 @@ mxq_status launch_gemm(mxq_format f, int dev, int sms, int64_t M, int64_t N, int
 
 bool valid_format(int f) { return f == MXQ_NVFP4 || f == MXQ_MXFP8 || f == MXQ_BF16; }
 
-// Byte layout shared by the activation workspace and weight storage:
-// [0,4) amax, [4,8) g, [256, 256+codes) codes, then the scales (256-aligned).
+// Byte layout of the weight storage and of the activation workspace:
+// [0,4) amax, [4,8) g, then (workspace only) the per-block amax partials at
+// [256, 256 + 4 * kMaxAmaxPartials), then the codes and the scales, each
+// 256-byte aligned.
+constexpr size_t kPartialsOff = 256;
+constexpr size_t kWorkspaceHeader = 8192;  // holds the partials
 struct QuantLayout {
   size_t codes_off, sf_off, total;
 };
-QuantLayout quant_layout(int64_t rows, int64_t k, mxq_format f) {
+QuantLayout quant_layout(int64_t rows, int64_t k, mxq_format f, size_t header = 256) {
   QuantLayout l;
-  l.codes_off = 256;
+  l.codes_off = header;
   l.sf_off = l.codes_off + static_cast<size_t>(pad_to(mxq_codes_bytes(rows, k, f), 256));
   l.total = l.sf_off + static_cast<size_t>(pad_to(mxq_sf_bytes(rows, k, f), 256));
   return l;
@@ -400,7 +420,7 @@ mxq_status mxq_quantize_nvfp4(const void* x_bf16, int64_t rows, int64_t k, int64
   int dev, sms;
   if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
   if (rows == 0 || k == 0) return MXQ_OK;
-  return launch_quant_nvfp4(x_bf16, rows, k, ld, amax_dev, codes, sf_swz, g_dev,
+  return launch_quant_nvfp4(x_bf16, rows, k, ld, amax_dev, 1, codes, sf_swz, g_dev, nullptr,
                             reinterpret_cast<cudaStream_t>(stream), sms);
 }
 
@@ -490,7 +510,7 @@ mxq_status mxq_weight_prepare(mxq_format f, const void* w_bf16, int64_t N, int64
     if (f == MXQ_NVFP4) {
       if ((st = launch_amax(w_bf16, N, K, K, amax, s, sms)) != MXQ_OK) return st;
       if (N > 0 && K > 0 &&
-          (st = launch_quant_nvfp4(w_bf16, N, K, K, amax, codes, sf, g, s, sms)) != MXQ_OK)
+          (st = launch_quant_nvfp4(w_bf16, N, K, K, amax, 1, codes, sf, g, nullptr, s, sms)) != MXQ_OK)
         return st;
       w.g_dev = g;
       w.amax_dev = amax;
@@ -518,7 +538,7 @@ int mxq_linear_path(const mxq_weight* w, int64_t M, const mxq_linear_opts* opts)
 size_t mxq_linear_workspace_bytes(int64_t M, int64_t K, mxq_format f) {
   if (f != MXQ_NVFP4 && f != MXQ_MXFP8) return 0;
   if (M < 0 || K < 0) return 0;
-  return quant_layout(M, K, f).total;
+  return quant_layout(M, K, f, kWorkspaceHeader).total;
 }
 
 mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* y_bf16, void* ws,
@@ -540,7 +560,7 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
   const mxq_format f = static_cast<mxq_format>(path);
   if (w->codes == nullptr || w->sf == nullptr) return MXQ_ERR_INVALID_ARG;
   if (f == MXQ_NVFP4 && w->g_dev == nullptr) return MXQ_ERR_INVALID_ARG;
-  const QuantLayout l = quant_layout(M, K, f);
+  const QuantLayout l = quant_layout(M, K, f, kWorkspaceHeader);
   if (ws == nullptr) return MXQ_ERR_INVALID_ARG;
   if (!aligned256(ws)) return MXQ_ERR_ALIGNMENT;
   if (ws_bytes < l.total) return MXQ_ERR_WORKSPACE;
@@ -553,8 +573,12 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
   uint8_t* codes = base + l.codes_off;
   uint8_t* sf = base + l.sf_off;
   if (f == MXQ_NVFP4) {
-    if ((st = launch_amax(x_bf16, M, K, K, amax, s, sms)) != MXQ_OK) return st;
-    if ((st = launch_quant_nvfp4(x_bf16, M, K, K, amax, codes, sf, g, s, sms)) != MXQ_OK) return st;
+    float* partials = reinterpret_cast<float*>(base + kPartialsOff);
+    int n_partials = 0;
+    if ((st = launch_amax_partials(x_bf16, M, K, K, partials, &n_partials, s, sms)) != MXQ_OK) return st;
+    if ((st = launch_quant_nvfp4(x_bf16, M, K, K, partials, n_partials, codes, sf, g, amax, s, sms)) !=
+        MXQ_OK)
+      return st;
   } else {
     if ((st = launch_quant_mxfp8(x_bf16, M, K, K, codes, sf, s, sms)) != MXQ_OK) return st;
   }

@@ -120,47 +120,67 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
 }
 
 // ------------------------------------------------------------------- amax
+// Work split: one warp per row (rows strided over all warps of the grid); a
+// lane owns every 32nd 16-byte vector of the row, four loads in flight.  No
+// integer division anywhere on the path.
 constexpr int kQuantThreads = 256;
 constexpr int kQuantUnroll = 4;
+constexpr int kMaxAmaxPartials = 1024;
 
-__global__ void __launch_bounds__(kQuantThreads) amax_kernel(const __nv_bfloat16* __restrict__ x,
-                                                             int64_t rows, int64_t k, int64_t ld,
-                                                             float* __restrict__ amax_out) {
-  const int64_t vpr = k >> 3;  // 16-byte vectors per row
-  const int64_t total = rows * vpr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kQuantThreads * kQuantUnroll;
-  float m = 0.0f;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kQuantThreads * kQuantUnroll + threadIdx.x;
-       base < total; base += stride) {
-    uint4 u[kQuantUnroll];
-#pragma unroll
-    for (int j = 0; j < kQuantUnroll; ++j) {
-      const int64_t t = base + j * kQuantThreads;
-      if (t < total) {
-        const int64_t r = t / vpr, v = t - r * vpr;
-        u[j] = ldg_nc_v4(x + r * ld + v * 8);
-      } else {
-        u[j] = make_uint4(0, 0, 0, 0);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kQuantUnroll; ++j) {
-      float f[8];
-      bf16x8_to_f32(u[j], f);
-      m = fmaxf(m, absmax8(f));
-    }
-  }
+__device__ __forceinline__ float warp_max(float m) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  __shared__ float warp_max[kQuantThreads / 32];
-  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+  return m;
+}
+
+// Block-wide max of `m` (every thread gets it).
+__device__ __forceinline__ float block_max(float m) {
+  __shared__ float s_max[kQuantThreads / 32];
+  m = warp_max(m);
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float b = warp_max[0];
+  if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float b = s_max[0];
 #pragma unroll
-    for (int i = 1; i < kQuantThreads / 32; ++i) b = fmaxf(b, warp_max[i]);
-    // non-negative floats order like their bit patterns
-    atomicMax(reinterpret_cast<unsigned int*>(amax_out), __float_as_uint(b));
+  for (int i = 1; i < kQuantThreads / 32; ++i) b = fmaxf(b, s_max[i]);
+  return b;
+}
+
+// max |x| of the rows this block's warps own, written to partial[blockIdx.x]
+// (or folded into *amax_atomic with atomicMax when partial is null).
+__global__ void __launch_bounds__(kQuantThreads) amax_kernel(const __nv_bfloat16* __restrict__ x,
+                                                             int rows, int k, int64_t ld,
+                                                             float* __restrict__ partial,
+                                                             float* __restrict__ amax_atomic) {
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (kQuantThreads / 32);
+  const int vpr = k >> 3;  // 16-byte vectors per row
+  float m = 0.0f;
+  for (int r = blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const __nv_bfloat16* row = x + static_cast<int64_t>(r) * ld;
+    for (int v0 = lane; v0 < vpr; v0 += 32 * kQuantUnroll) {
+      uint4 u[kQuantUnroll];
+#pragma unroll
+      for (int j = 0; j < kQuantUnroll; ++j) {
+        const int v = v0 + 32 * j;
+        u[j] = v < vpr ? ldg_nc_v4(row + v * 8) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < kQuantUnroll; ++j) {
+        float f[8];
+        bf16x8_to_f32(u[j], f);
+        m = fmaxf(m, absmax8(f));
+      }
+    }
+  }
+  m = block_max(m);
+  if (threadIdx.x == 0) {
+    if (partial != nullptr) {
+      partial[blockIdx.x] = m;
+    } else {
+      // non-negative floats order like their bit patterns
+      atomicMax(reinterpret_cast<unsigned int*>(amax_atomic), __float_as_uint(m));
+    }
   }
 }
 
@@ -170,109 +190,111 @@ __device__ __forceinline__ float nvfp4_global_scale(float amax) {
 }
 
 // Zero the scale bytes of padding rows [rows, pad128(rows)).
-__device__ __forceinline__ void zero_sf_padding(uint8_t* __restrict__ sf, int64_t rows, int64_t c,
-                                                int64_t tid, int64_t nthreads) {
-  const int64_t rp = (rows + 127) / 128 * 128;
-  const int64_t total = (rp - rows) * c;
-  const int64_t c4 = c >> 2;
-  for (int64_t t = tid; t < total; t += nthreads) {
-    const int64_t r = rows + t / c, cc = t % c;
+__device__ __forceinline__ void zero_sf_padding(uint8_t* __restrict__ sf, int rows, int c) {
+  const int rp = (rows + 127) / 128 * 128;
+  const int total = (rp - rows) * c;
+  const int c4 = c >> 2;
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < total; t += gridDim.x * blockDim.x) {
+    const int r = rows + t / c, cc = t - (t / c) * c;
     sf[sf_offset(r, cc, c4)] = 0;
   }
 }
 
+// amax_in: n_amax values whose max is the tensor's amax (1 value, or the
+// per-block partials of amax_kernel).
 __global__ void __launch_bounds__(kQuantThreads)
-    quantize_nvfp4_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
-                          const float* __restrict__ amax_in, uint8_t* __restrict__ codes,
-                          uint8_t* __restrict__ sf, float* __restrict__ g_out) {
-  const float g = nvfp4_global_scale(*amax_in);
+    quantize_nvfp4_kernel(const __nv_bfloat16* __restrict__ x, int rows, int k, int64_t ld,
+                          const float* __restrict__ amax_in, int n_amax, uint8_t* __restrict__ codes,
+                          uint8_t* __restrict__ sf, float* __restrict__ g_out,
+                          float* __restrict__ amax_out) {
+  float a = 0.0f;
+  for (int i = threadIdx.x; i < n_amax; i += kQuantThreads) a = fmaxf(a, amax_in[i]);
+  a = block_max(a);
+  const float g = nvfp4_global_scale(a);
   const float six_g = 6.0f * g;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
-  const int64_t vpr = k >> 3;
-  const int64_t total = rows * vpr;  // even: k is a multiple of 16
-  const int64_t c4 = k >> 6;         // 4-column scale groups per row
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kQuantThreads * kQuantUnroll;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kQuantThreads * kQuantUnroll + threadIdx.x;
-       base - threadIdx.x < total; base += stride) {
-    uint4 u[kQuantUnroll];
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *g_out = g;
+    if (amax_out != nullptr) *amax_out = a;
+  }
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (kQuantThreads / 32);
+  const int vpr = k >> 3;  // even: k is a multiple of 16
+  const int c4 = k >> 6;   // 4-column scale groups per row
+  for (int r = blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const __nv_bfloat16* row = x + static_cast<int64_t>(r) * ld;
+    uint32_t* crow = reinterpret_cast<uint32_t*>(codes + static_cast<int64_t>(r) * (k >> 1));
+    for (int v0 = lane; v0 - lane < vpr; v0 += 32 * kQuantUnroll) {
+      uint4 u[kQuantUnroll];
 #pragma unroll
-    for (int j = 0; j < kQuantUnroll; ++j) {
-      const int64_t t = base + j * kQuantThreads;
-      if (t < total) {
-        const int64_t r = t / vpr, v = t - r * vpr;
-        u[j] = ldg_nc_v4(x + r * ld + v * 8);
-      } else {
-        u[j] = make_uint4(0, 0, 0, 0);
+      for (int j = 0; j < kQuantUnroll; ++j) {
+        const int v = v0 + 32 * j;
+        u[j] = v < vpr ? ldg_nc_v4(row + v * 8) : make_uint4(0, 0, 0, 0);
       }
-    }
 #pragma unroll
-    for (int j = 0; j < kQuantUnroll; ++j) {
-      const int64_t t = base + j * kQuantThreads;
-      float f[8];
-      bf16x8_to_f32(u[j], f);
-      float bmax = absmax8(f);
-      bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));  // 16-element block
-      const uint32_t sfc = cvt_e4m3x2(bmax / six_g, 0.0f) & 0xFFu;
-      const float s = e4m3_value(sfc) * g;
-      const float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
+      for (int j = 0; j < kQuantUnroll; ++j) {
+        const int v = v0 + 32 * j;
+        if (v - lane >= vpr) break;  // warp-uniform
+        float f[8];
+        bf16x8_to_f32(u[j], f);
+        float bmax = absmax8(f);
+        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));  // 16-element block
+        const uint32_t sfc = cvt_e4m3x2(bmax / six_g, 0.0f) & 0xFFu;
+        const float s = e4m3_value(sfc) * g;
+        const float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) f[i] = f[i] * inv;
-      const uint32_t packed = cvt_e2m1x8(f);
-      if (t < total) {
-        const int64_t r = t / vpr, v = t - r * vpr;
-        *reinterpret_cast<uint32_t*>(codes + r * (k >> 1) + v * 4) = packed;
-        if ((v & 1) == 0) sf[sf_offset(r, v >> 1, c4)] = static_cast<uint8_t>(sfc);
+        for (int i = 0; i < 8; ++i) f[i] = f[i] * inv;
+        const uint32_t packed = cvt_e2m1x8(f);
+        if (v < vpr) {
+          crow[v] = packed;
+          if ((v & 1) == 0) sf[sf_offset(r, v >> 1, c4)] = static_cast<uint8_t>(sfc);
+        }
       }
     }
   }
-  zero_sf_padding(sf, rows, k >> 4, static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x,
-                  static_cast<int64_t>(gridDim.x) * kQuantThreads);
+  zero_sf_padding(sf, rows, k >> 4);
 }
 
 // -------------------------------------------------------------- MXFP8
 __global__ void __launch_bounds__(kQuantThreads)
-    quantize_mxfp8_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t k, int64_t ld,
+    quantize_mxfp8_kernel(const __nv_bfloat16* __restrict__ x, int rows, int k, int64_t ld,
                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
-  const int64_t vpr = k >> 3;
-  const int64_t total = rows * vpr;  // multiple of 4: k is a multiple of 32
-  const int64_t c4 = k >> 7;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kQuantThreads * kQuantUnroll;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kQuantThreads * kQuantUnroll + threadIdx.x;
-       base - threadIdx.x < total; base += stride) {
-    uint4 u[kQuantUnroll];
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (kQuantThreads / 32);
+  const int vpr = k >> 3;  // multiple of 16: k is a multiple of 128
+  const int c4 = k >> 7;
+  for (int r = blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const __nv_bfloat16* row = x + static_cast<int64_t>(r) * ld;
+    uint2* crow = reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * k);
+    for (int v0 = lane; v0 - lane < vpr; v0 += 32 * kQuantUnroll) {
+      uint4 u[kQuantUnroll];
 #pragma unroll
-    for (int j = 0; j < kQuantUnroll; ++j) {
-      const int64_t t = base + j * kQuantThreads;
-      if (t < total) {
-        const int64_t r = t / vpr, v = t - r * vpr;
-        u[j] = ldg_nc_v4(x + r * ld + v * 8);
-      } else {
-        u[j] = make_uint4(0, 0, 0, 0);
+      for (int j = 0; j < kQuantUnroll; ++j) {
+        const int v = v0 + 32 * j;
+        u[j] = v < vpr ? ldg_nc_v4(row + v * 8) : make_uint4(0, 0, 0, 0);
       }
-    }
 #pragma unroll
-    for (int j = 0; j < kQuantUnroll; ++j) {
-      const int64_t t = base + j * kQuantThreads;
-      float f[8];
-      bf16x8_to_f32(u[j], f);
-      float bmax = absmax8(f);
-      bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
-      bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));  // 32-element block
-      int X = -127;
-      if (bmax > 0.0f) X = min(max(floor_log2_f32(bmax) - 8, -127), 127);
-      const float mult = exp2_int(-X);
-      uint2 out;
-      out.x = cvt_e4m3x2(f[0] * mult, f[1] * mult) | (cvt_e4m3x2(f[2] * mult, f[3] * mult) << 16);
-      out.y = cvt_e4m3x2(f[4] * mult, f[5] * mult) | (cvt_e4m3x2(f[6] * mult, f[7] * mult) << 16);
-      if (t < total) {
-        const int64_t r = t / vpr, v = t - r * vpr;
-        *reinterpret_cast<uint2*>(codes + r * k + v * 8) = out;
-        if ((v & 3) == 0) sf[sf_offset(r, v >> 2, c4)] = static_cast<uint8_t>(X + 127);
+      for (int j = 0; j < kQuantUnroll; ++j) {
+        const int v = v0 + 32 * j;
+        if (v - lane >= vpr) break;  // warp-uniform
+        float f[8];
+        bf16x8_to_f32(u[j], f);
+        float bmax = absmax8(f);
+        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
+        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));  // 32-element block
+        int X = -127;
+        if (bmax > 0.0f) X = min(max(floor_log2_f32(bmax) - 8, -127), 127);
+        const float mult = exp2_int(-X);
+        uint2 out;
+        out.x = cvt_e4m3x2(f[0] * mult, f[1] * mult) | (cvt_e4m3x2(f[2] * mult, f[3] * mult) << 16);
+        out.y = cvt_e4m3x2(f[4] * mult, f[5] * mult) | (cvt_e4m3x2(f[6] * mult, f[7] * mult) << 16);
+        if (v < vpr) {
+          crow[v] = out;
+          if ((v & 3) == 0) sf[sf_offset(r, v >> 2, c4)] = static_cast<uint8_t>(X + 127);
+        }
       }
     }
   }
-  zero_sf_padding(sf, rows, k >> 5, static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x,
-                  static_cast<int64_t>(gridDim.x) * kQuantThreads);
+  zero_sf_padding(sf, rows, k >> 5);
 }
 
 // ----------------------------------------------- conversion check kernel
