@@ -167,6 +167,10 @@ __global__ void __launch_bounds__(GemmCfg<F, BN>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // everything above overlaps the previous kernel's tail; A, its scales and
+  // the per-tensor scales are that kernel's output
+  grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer

@@ -183,6 +183,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
   cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // everything above overlaps the previous kernel's tail; A, its scales and
+  // the per-tensor scales are that kernel's output
+  grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ A/B producer

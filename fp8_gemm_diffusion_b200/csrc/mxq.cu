@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/mxq.h"
 #include "gemm.cuh"
@@ -133,16 +134,34 @@ mxq_status check_bf16_matrix(const void* x, int64_t rows, int64_t k, int64_t ld)
 }
 
 // ----------------------------------------------------------------- launches
+// Every kernel is launched with programmatic stream serialization: it may
+// start while the previous kernel of the stream finishes, and waits
+// (griddepcontrol.wait) before reading anything that kernel wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // amax into one fp32 (zeroed first, then atomicMax of every block's maximum).
 mxq_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ld, float* amax,
                        cudaStream_t s, int sms) {
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
   if (e != cudaSuccess) return cuda_fail(e);
   if (rows == 0 || k == 0) return MXQ_OK;
-  mxq::amax_kernel<<<quant_grid(rows, sms), mxq::kQuantThreads, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<int>(rows), static_cast<int>(k), ld, nullptr,
-      amax);
-  e = cudaGetLastError();
+  e = launch_pdl(mxq::amax_kernel, dim3(quant_grid(rows, sms)), dim3(mxq::kQuantThreads), 0, s,
+                 static_cast<const __nv_bfloat16*>(x), static_cast<int>(rows), static_cast<int>(k), ld,
+                 static_cast<float*>(nullptr), amax);
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
@@ -150,30 +169,28 @@ mxq_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ld, float
 mxq_status launch_amax_partials(const void* x, int64_t rows, int64_t k, int64_t ld, float* partials,
                                 int* n_partials, cudaStream_t s, int sms) {
   const int grid = quant_grid(rows, sms);
-  mxq::amax_kernel<<<grid, mxq::kQuantThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                                       static_cast<int>(rows), static_cast<int>(k),
-                                                       ld, partials, nullptr);
+  cudaError_t e = launch_pdl(mxq::amax_kernel, dim3(grid), dim3(mxq::kQuantThreads), 0, s,
+                             static_cast<const __nv_bfloat16*>(x), static_cast<int>(rows),
+                             static_cast<int>(k), ld, partials, static_cast<float*>(nullptr));
   *n_partials = grid;
-  cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
 mxq_status launch_quant_nvfp4(const void* x, int64_t rows, int64_t k, int64_t ld,
                               const float* amax_vals, int n_amax, uint8_t* codes, uint8_t* sf,
                               float* g, float* amax_out, cudaStream_t s, int sms) {
-  mxq::quantize_nvfp4_kernel<<<quant_grid(rows, sms), mxq::kQuantThreads, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<int>(rows), static_cast<int>(k), ld,
-      amax_vals, n_amax, codes, sf, g, amax_out);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(mxq::quantize_nvfp4_kernel, dim3(quant_grid(rows, sms)),
+                             dim3(mxq::kQuantThreads), 0, s, static_cast<const __nv_bfloat16*>(x),
+                             static_cast<int>(rows), static_cast<int>(k), ld, amax_vals, n_amax, codes,
+                             sf, g, amax_out);
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
 mxq_status launch_quant_mxfp8(const void* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
                               uint8_t* sf, cudaStream_t s, int sms) {
-  mxq::quantize_mxfp8_kernel<<<quant_grid(rows, sms), mxq::kQuantThreads, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<int>(rows), static_cast<int>(k), ld, codes,
-      sf);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(mxq::quantize_mxfp8_kernel, dim3(quant_grid(rows, sms)),
+                             dim3(mxq::kQuantThreads), 0, s, static_cast<const __nv_bfloat16*>(x),
+                             static_cast<int>(rows), static_cast<int>(k), ld, codes, sf);
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
@@ -222,8 +239,7 @@ mxq_status launch_gemm_bn(int dev, int sms, int slot, int64_t M, int64_t N, int6
   args.bias = static_cast<const __nv_bfloat16*>(bias);
   const int64_t tiles = ((M + C::BM - 1) / C::BM) * ((N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, ty, args);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, ta, tb, ty, args);
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
@@ -281,8 +297,8 @@ mxq_status launch_gemm_pair(int dev, int sms, int slot, int64_t M, int64_t N, in
   const int64_t tiles = ((M + C::BM - 1) / C::BM) * ((N + BN - 1) / BN);
   const int64_t pairs = sms / 2;
   const int grid = 2 * static_cast<int>(tiles < pairs ? tiles : pairs);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, tsa, tsb, ty, args);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, ta, tb, tsa, tsb, ty,
+                             args);
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 

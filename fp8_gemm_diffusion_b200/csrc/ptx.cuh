@@ -414,3 +414,20 @@ __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint32_t a, ui
 }
 
 }  // namespace mxq
+
+namespace mxq {
+
+// Programmatic dependent launch: wait until the preceding kernel of the stream
+// has completed and its memory is visible (a no-op without a predecessor or
+// when launched without the programmatic attribute) ...
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// ... and allow the next kernel of the stream to start launching (its own
+// grid_dep_wait still orders its dependent reads after this grid's end).
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace mxq

@@ -152,6 +152,8 @@ __global__ void __launch_bounds__(kQuantThreads) amax_kernel(const __nv_bfloat16
                                                              int rows, int k, int64_t ld,
                                                              float* __restrict__ partial,
                                                              float* __restrict__ amax_atomic) {
+  grid_dep_wait();  // x may be the previous kernel's output
+  grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (kQuantThreads / 32);
   const int vpr = k >> 3;  // 16-byte vectors per row
@@ -207,6 +209,8 @@ __global__ void __launch_bounds__(kQuantThreads)
                           const float* __restrict__ amax_in, int n_amax, uint8_t* __restrict__ codes,
                           uint8_t* __restrict__ sf, float* __restrict__ g_out,
                           float* __restrict__ amax_out) {
+  grid_dep_wait();  // the amax (partials) comes from the previous kernel
+  grid_dep_launch();
   float a = 0.0f;
   for (int i = threadIdx.x; i < n_amax; i += kQuantThreads) a = fmaxf(a, amax_in[i]);
   a = block_max(a);
@@ -258,6 +262,8 @@ __global__ void __launch_bounds__(kQuantThreads)
 __global__ void __launch_bounds__(kQuantThreads)
     quantize_mxfp8_kernel(const __nv_bfloat16* __restrict__ x, int rows, int k, int64_t ld,
                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (kQuantThreads / 32);
   const int vpr = k >> 3;  // multiple of 16: k is a multiple of 128
