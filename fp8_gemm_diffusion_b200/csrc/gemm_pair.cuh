@@ -73,10 +73,16 @@ struct PairCfg {
   static constexpr int TMEM_COLS = 512;
   // one scale set per A/B stage: a set is free when its stage is (same commit)
   static constexpr int NS_FIT = SCALED ? (TMEM_COLS - BN) / SF_SET_COLS : 64;
-  static constexpr int SF_WARPS = 4;   // one per tensor-memory sub-partition
-  static constexpr int EPI_WARPS = 4;  // one per sub-partition
-  static constexpr int EPI_BATCHES = BN / 128;
-  static constexpr int EPI_BYTES = EPI_WARPS * 32 * 128 * 2;  // one 128-column batch per warp
+  // warp roles, one warpgroup each for (producer, MMA, scale loader, spare),
+  // the scale writers and the two halves of the epilogue
+  static constexpr int SF_WARP0 = 4;   // warps 4-7, one per tensor-memory sub-partition
+  static constexpr int SF_WARPS = 4;
+  static constexpr int EPI_WARP0 = 8;  // warps 8-15: sub-partition warp % 4, column half (warp / 4) % 2
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_COLS = BN / 2;   // accumulator columns per epilogue warp
+  static constexpr int EPI_BYTES = EPI_WARPS * 32 * 64 * 2;  // a 32 x 64 staging sub-tile per warp
+  // registers: launched with 65536 / 512 = 128 per thread, then rebalanced
+  static constexpr int REGS_CTRL = 56, REGS_SFW = 80, REGS_EPI = 184;
   static constexpr int BAR_BYTES = 512;
   static constexpr int STAGES_FIT =
       (232448 - 1024 - BAR_BYTES - EPI_BYTES - SF_SLOTS * SF_SLOT_BYTES) / STAGE_BYTES;
@@ -86,7 +92,8 @@ struct PairCfg {
   static_assert(STAGES >= 2, "shared / tensor memory");
   static constexpr int SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + EPI_BYTES + BAR_BYTES;
-  static constexpr int THREADS = 32 * (3 + SF_WARPS + EPI_WARPS);
+  static constexpr int THREADS = 512;
+  static_assert(128 * (REGS_CTRL + REGS_SFW) + 256 * REGS_EPI <= 65536, "register split");
 };
 
 // Instruction descriptor of an M=256 (pair) MMA; fields as in make_idesc.
@@ -188,6 +195,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
   grid_dep_wait();
   grid_dep_launch();
 
+  // Registers move from the control and scale-writer warpgroups to the
+  // epilogue: each warpgroup's setmaxnreg opens its role's code.
+  if (warp < C::SF_WARP0) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_CTRL));
   if (warp == 0) {
     // ------------------------------------------------------------ A/B producer
     if (lane == 0) {
@@ -309,7 +320,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         }
       }
     }
-  } else if (warp < 3 + C::SF_WARPS) {
+  } else if (warp == 3) {
+    // spare warp of the control warpgroup
+  }
+  } else if (warp < C::EPI_WARP0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_SFW));
     // ------------------------------------------------ scale factors -> TMEM
     // Each warp writes the 32 lanes of its sub-partition: lane l receives row l
     // of every 512-byte scale chunk of the stage (16 bytes = 4 columns), the
@@ -367,9 +382,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       }
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_EPI));
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // tensor-memory sub-partition = 32-row slice
-    const uint32_t stage_buf = epi_base + (warp - 3 - C::SF_WARPS) * (32 * 128 * 2);
+    const int q = warp & 3;          // tensor-memory sub-partition = 32-row slice
+    const int h = (warp >> 2) & 1;   // column half of the tile
+    const uint32_t stage_buf = epi_base + (warp - C::EPI_WARP0) * (32 * 64 * 2);
     const uint32_t leader_tempty = map_to_cta(tempty_bar, 0);
     float alpha = 1.0f;
     if constexpr (F == Fmt::NVFP4) alpha = (*args.a_g) * (*args.b_g);
@@ -398,54 +415,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       }
       if (!mbar_wait_bounded(tfull_bar, i_tile & 1)) break;
       tc_fence_after();
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-#pragma unroll 1
-      for (int bt = 0; bt < C::EPI_BATCHES; ++bt) {
-        // 128 accumulator columns at once; the last batch releases the accumulator
-        uint32_t r[128];
+      // all of this warp's accumulator columns into registers, then release the accumulator
+      uint32_t r[C::EPI_COLS];
+      const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + h * C::EPI_COLS;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x32_nowait(t_row + bt * 128 + g * 32, r + 32 * g);
-        tc_wait_ld();
+      for (int g = 0; g < C::EPI_COLS / 32; ++g) tmem_ld_32x32b_x32_nowait(t_cols + g * 32, r + 32 * g);
+      tc_wait_ld();
 #pragma unroll
-        for (int g = 0; g < 4; ++g) reg_fence32(r + 32 * g);
-        if (bt == C::EPI_BATCHES - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_remote(leader_tempty);  // accumulator may be overwritten
-        }
-        if (lane == 0) bulk_wait_group_read<0>();  // previous batch's stores have read the staging
+      for (int g = 0; g < C::EPI_COLS / 32; ++g) reg_fence32(r + 32 * g);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(leader_tempty);  // accumulator may be overwritten
+      const int col_w = nt * BN + h * C::EPI_COLS;  // first column of this warp
+#pragma unroll
+      for (int sub = 0; sub < C::EPI_COLS / 64; ++sub) {
+        if (lane == 0) bulk_wait_group_read<0>();  // the staging sub-tile is free again
         __syncwarp();
-        const int col_base = nt * BN + bt * 128;
-        // 16 groups of 8 columns: bias (8 bf16), alpha * acc + bias, bf16, one 16-byte store
-        // into the staging (two sub-tiles of 32 rows x 64 columns, 128-byte swizzle)
+        // 8 groups of 8 columns: alpha * acc + bias, bf16, one 16-byte store each
+        // into a 32 x 64 staging sub-tile (128 B rows, 128-byte swizzle)
 #pragma unroll
-        for (int j16 = 0; j16 < 16; ++j16) {
-          uint32_t bw[4];  // bias of columns [8 * (16 bt + j16), +8) from the lane holding them
+        for (int j = 0; j < 8; ++j) {
+          const int grp = h * (C::EPI_COLS / 8) + sub * 8 + j;  // 8-column group within the tile
+          uint32_t bw[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) bw[e] = __shfl_sync(0xffffffffu, bias_l[e], bt * 16 + j16);
+          for (int e = 0; e < 4; ++e) bw[e] = __shfl_sync(0xffffffffu, bias_l[e], grp);
           uint32_t pk[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            float v0 = __uint_as_float(r[8 * j16 + 2 * e]), v1 = __uint_as_float(r[8 * j16 + 2 * e + 1]);
+            const int c = sub * 64 + j * 8 + 2 * e;
+            float v0 = __uint_as_float(r[c]), v1 = __uint_as_float(r[c + 1]);
             if constexpr (F == Fmt::NVFP4) { v0 *= alpha; v1 *= alpha; }
             v0 += __uint_as_float(bw[e] << 16);
             v1 += __uint_as_float(bw[e] & 0xFFFF0000u);
             const __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
             pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
           }
-          const int j = j16 & 7;  // 16-byte chunk within the 128-byte row
-          const uint32_t addr = stage_buf + (j16 >> 3) * 4096 + lane * 128 + ((j ^ (lane & 7)) << 4);
+          const uint32_t addr = stage_buf + lane * 128 + ((j ^ (lane & 7)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]),
                        "r"(pk[2]), "r"(pk[3])
                        : "memory");
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && row0 < M) {
-          for (int k = 0; k < 2; ++k) {
-            const int x = col_base + 64 * k;
-            if (x < N) tma_store_2d(&tmap_y, stage_buf + k * 4096, x, row0);
-          }
+        const int x = col_w + sub * 64;
+        if (lane == 0 && row0 < M && x < N) {
+          tma_store_2d(&tmap_y, stage_buf, x, row0);
           bulk_commit_group();
         }
       }
