@@ -9,25 +9,25 @@
 // tensor memory.  Per CTA this halves the operand traffic of a 128 x BN tile
 // and the pair MMA runs the tensor cores at a higher rate than M=128 MMAs.
 //
-// Roles (both CTAs):
+// Roles (both CTAs; 16 warps, registers rebalanced per warpgroup):
 //   warp 0      A/B producer: each stage's 128 rows of A and BN/2 rows of B
 //               into this CTA's ring; completions land on the even CTA's full
 //               barrier (cta_group::2 loads, no multicast).
 //   warp 1      tensor memory (cta_group::2 allocation); on the even CTA one
 //               lane issues the MMAs and commits to both CTAs' barriers
-//               (multicast commit): A/B stage free, scale set free, and
-//               accumulator full.
+//               (multicast commit): A/B stage free (the scale set that the
+//               stage read is free from then on too) and accumulator full.
 //   warp 2      scale loader: the scale chunks of each stage (A's 128 rows and
 //               all BN columns of B: each CTA's tensor memory needs B's) into
 //               a separate ring that runs ahead of the A/B ring.
-//   warps 3-6   scale writers, one per tensor-memory sub-partition: chunk rows
-//               from shared memory into a per-stage set of tensor-memory
+//   warps 4-7   scale writers, one per tensor-memory sub-partition: chunk rows
+//               from shared memory into one of NS sets of tensor-memory
 //               columns with tcgen05.st, so no tcgen05.cp sits between MMAs.
-//               They run up to NS stages ahead of the MMAs.
-//   warps 7-10  epilogue, one per sub-partition: 128 accumulator columns per
-//               batch into registers, release the accumulator after the last
-//               batch, then alpha, bias, bf16, 128-byte swizzled staging and
-//               TMA stores.
+//   warps 8-15  epilogue, sub-partition warp % 4, column half (warp / 4) % 2:
+//               the warp's accumulator columns into registers, release of the
+//               accumulator, then alpha, bias, bf16, 64-byte swizzled staging
+//               and TMA stores of 32 x 32 sub-tiles.
+// Tiles are visited along the smaller operand first (pair_tile_coords).
 // Every wait is bounded (ptx.cuh); a timed-out role stops, loads and MMAs in
 // flight are drained, and both CTAs free tensor memory together.
 #pragma once
@@ -71,7 +71,8 @@ struct PairCfg {
   static constexpr int SF_COL = BN;
   static constexpr int SFB_OFF = SF_CHUNKS * 4;
   static constexpr int TMEM_COLS = 512;
-  // one scale set per A/B stage: a set is free when its stage is (same commit)
+  // scale sets in tensor memory: stage k uses set k % NS, free again when the
+  // MMAs of stage k - NS have completed (that stage's A/B commit)
   static constexpr int NS_FIT = SCALED ? (TMEM_COLS - BN) / SF_SET_COLS : 64;
   // warp roles, one warpgroup each for (producer, MMA, scale loader, spare),
   // the scale writers and the two halves of the epilogue
@@ -80,15 +81,15 @@ struct PairCfg {
   static constexpr int EPI_WARP0 = 8;  // warps 8-15: sub-partition warp % 4, column half (warp / 4) % 2
   static constexpr int EPI_WARPS = 8;
   static constexpr int EPI_COLS = BN / 2;   // accumulator columns per epilogue warp
-  static constexpr int EPI_BYTES = EPI_WARPS * 32 * 64 * 2;  // a 32 x 64 staging sub-tile per warp
+  static constexpr int EPI_SUB = 32;        // staging sub-tile: 32 rows x 32 columns (64-byte rows)
+  static constexpr int EPI_BYTES = EPI_WARPS * 32 * EPI_SUB * 2;
   // registers: launched with 65536 / 512 = 128 per thread, then rebalanced
   static constexpr int REGS_CTRL = 56, REGS_SFW = 80, REGS_EPI = 184;
   static constexpr int BAR_BYTES = 512;
   static constexpr int STAGES_FIT =
       (232448 - 1024 - BAR_BYTES - EPI_BYTES - SF_SLOTS * SF_SLOT_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES_MIN = STAGES_FIT < NS_FIT ? STAGES_FIT : NS_FIT;
-  static constexpr int STAGES = STAGES_MIN > 6 ? 6 : STAGES_MIN;
-  static constexpr int NS = STAGES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int NS = NS_FIT < STAGES ? NS_FIT : STAGES;
   static_assert(STAGES >= 2, "shared / tensor memory");
   static constexpr int SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + EPI_BYTES + BAR_BYTES;
@@ -107,6 +108,20 @@ __device__ __forceinline__ uint32_t make_idesc_pair(int n, uint32_t sf_id) {
     return (sf_id << 4) | n_field | (1u << 23) | m_field | (sf_id << 29);
   } else {
     return (1u << 4) | (1u << 7) | (1u << 10) | n_field | m_field;
+  }
+}
+
+// Tile order: tiles run along the dimension of the smaller operand first, so
+// the pairs working at the same time share all of that operand (it stays in
+// L2) and only a few strips of the larger one, which HBM then delivers once.
+__device__ __forceinline__ void pair_tile_coords(int tile, int m_tiles, int n_tiles, bool n_fast,
+                                                 int& mt, int& nt) {
+  if (n_fast) {
+    mt = tile / n_tiles;
+    nt = tile - mt * n_tiles;
+  } else {
+    nt = tile / m_tiles;
+    mt = tile - nt * m_tiles;
   }
 }
 
@@ -152,6 +167,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
   const int m_tiles = (M + C::BM - 1) / C::BM;
   const int n_tiles = (N + BN - 1) / BN;
   const int num_tiles = m_tiles * n_tiles;
+  const bool n_fast = N < M;  // B is the smaller operand
   const int num_kb = (K + C::K_STAGE - 1) / C::K_STAGE;
   const int sf_c4 = F == Fmt::NVFP4 ? K / 64 : (F == Fmt::MXFP8 ? K / 128 : 0);
   const int pair = blockIdx.x >> 1;
@@ -209,7 +225,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       const int b_row_off = static_cast<int>(rank) * C::BN_CTA;
       constexpr int KX = C::ROW_BYTES / (F == Fmt::BF16 ? 2 : 1);  // K coordinate step per stage
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int nt = tile / m_tiles, mt = tile - nt * m_tiles;
+        int mt, nt;
+        pair_tile_coords(tile, m_tiles, n_tiles, n_fast, mt, nt);
         const int a_row = mt * C::BM + a_row_off, b_row = nt * BN + b_row_off;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u)) { ok = false; break; }
@@ -234,15 +251,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
     // ------------------------------------------------------------ MMA issuer
     // (one thread: keep the per-stage work to a few instructions)
     if (lane == 0 && rank == 0) {
-      int s = 0;
-      uint32_t ph = 0, acc_ph = 0;
+      int s = 0, n = 0;
+      uint32_t ph = 0, nph = 0, acc_ph = 0;
       bool ok = true;
       const uint64_t adesc0 = desc_kmajor_sw128(base);
       const uint64_t bdesc0 = desc_kmajor_sw128(base + C::A_BYTES);
       constexpr uint64_t DSTEP = C::STAGE_BYTES >> 4;  // descriptor start-address step per stage
       const uint32_t idesc = make_idesc_pair<F>(BN, 0);
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int nt = tile / m_tiles;
+        int mt, nt;
+        pair_tile_coords(tile, m_tiles, n_tiles, n_fast, mt, nt);
         const uint32_t sfb_shift = ((nt * BN) & 127) >> 5;
         // the accumulator is single-buffered: wait until the epilogue has read the last tile
         if (!mbar_wait_bounded(tempty_bar, acc_ph ^ 1u)) { ok = false; break; }
@@ -250,10 +268,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         tc_fence_after();
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(full_bar(s), ph)) { ok = false; break; }
-          if (C::SCALED && !mbar_wait_bounded(sf_ready_bar(s), ph)) { ok = false; break; }
+          if (C::SCALED && !mbar_wait_bounded(sf_ready_bar(n), nph)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = adesc0 + DSTEP * s, bdesc = bdesc0 + DSTEP * s;
-          const uint32_t sf = tmem_base + C::SF_COL + s * C::SF_SET_COLS;
+          const uint32_t sf = tmem_base + C::SF_COL + n * C::SF_SET_COLS;
           int nmma = C::MMAS;
           if constexpr (F == Fmt::NVFP4) {
             if (kb == num_kb - 1) nmma = K / 64 - kb * C::MMAS;  // K % 256 != 0: partial last stage
@@ -276,8 +294,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
               }
             }
           }
-          tc_commit_pair(empty_bar(s));  // frees A/B stage s and scale set s
+          tc_commit_pair(empty_bar(s));  // frees A/B stage s (and scale set n, NS stages on)
           if (++s == S) { s = 0; ph ^= 1u; }
+          if (++n == NS) { n = 0; nph ^= 1u; }
         }
         if (!ok) break;
         tc_commit_pair(tfull_bar);
@@ -295,7 +314,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       uint32_t ph = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int nt = tile / m_tiles, mt = tile - nt * m_tiles;
+        int mt, nt;
+        pair_tile_coords(tile, m_tiles, n_tiles, n_fast, mt, nt);
         // 512-byte chunk (row block rb, 4-column group kc) is 256-byte row 2*(rb*sf_c4+kc)
         const int ya = 2 * (mt * 2 + static_cast<int>(rank)) * sf_c4;
         const int yb = 2 * (nt * BN / 128) * sf_c4;
@@ -334,8 +354,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       const uint32_t q = static_cast<uint32_t>(warp & 3);
       const uint32_t leader_ready0 = map_to_cta(sf_ready_bar(0), 0);
       constexpr int NCH = C::SF_CHUNKS * (1 + C::NRB);  // A chunks, then B chunks
-      int r = 0, n = 0;
-      uint32_t rph = 0, nph = 0;
+      int r = 0, n = 0, js = 0;
+      uint32_t rph = 0, jph = 0;
       for (int g = 0; g < total_kb; ++g) {
         if (!mbar_wait_bounded(sf_full_bar(r), rph)) break;
         const uint32_t slot = sf_base + r * C::SF_SLOT_BYTES;
@@ -356,8 +376,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(sf_empty_bar(r));  // slot read: the loader may refill it
-        // the set is free once the MMAs of stage g - NS have completed
-        if (g >= NS && !mbar_wait_bounded(empty_bar(n), nph ^ 1u)) break;
+        // set n is free once the MMAs of stage j = g - NS (A/B slot js, that
+        // slot's completion number j / S) have completed
+        if (g >= NS) {
+          if (!mbar_wait_bounded(empty_bar(js), jph)) break;
+          if (++js == S) { js = 0; jph ^= 1u; }
+        }
         tc_fence_after();
         const uint32_t t = tmem_base + (q * 32u << 16) + C::SF_COL + n * C::SF_SET_COLS;
         if constexpr (NCH * 4 % 16 == 0) {
@@ -378,7 +402,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(leader_ready0 + 8u * n);
         if (++r == R) { r = 0; rph ^= 1u; }
-        if (++n == NS) { n = 0; nph ^= 1u; }
+        if (++n == NS) n = 0;
       }
     }
   } else {
@@ -386,14 +410,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;          // tensor-memory sub-partition = 32-row slice
     const int h = (warp >> 2) & 1;   // column half of the tile
-    const uint32_t stage_buf = epi_base + (warp - C::EPI_WARP0) * (32 * 64 * 2);
+    const uint32_t stage_buf = epi_base + (warp - C::EPI_WARP0) * (32 * C::EPI_SUB * 2);
     const uint32_t leader_tempty = map_to_cta(tempty_bar, 0);
     float alpha = 1.0f;
     if constexpr (F == Fmt::NVFP4) alpha = (*args.a_g) * (*args.b_g);
     const bool bias_vec = args.bias != nullptr && (reinterpret_cast<uintptr_t>(args.bias) & 15u) == 0;
     for (int i_tile = 0; i_tile < my_tiles; ++i_tile) {
       const int tile = pair + i_tile * num_pairs;
-      const int mt = tile % m_tiles, nt = tile / m_tiles;
+      int mt, nt;
+      pair_tile_coords(tile, m_tiles, n_tiles, n_fast, mt, nt);
       const int row0 = mt * C::BM + static_cast<int>(rank) * C::BM_CTA + q * 32;
       // the tile's bias, prefetched before the accumulator is ready: lane l holds
       // columns [8l, 8l + 8) of the tile as four packed bf16 pairs
@@ -428,21 +453,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       if (lane == 0) mbar_arrive_remote(leader_tempty);  // accumulator may be overwritten
       const int col_w = nt * BN + h * C::EPI_COLS;  // first column of this warp
 #pragma unroll
-      for (int sub = 0; sub < C::EPI_COLS / 64; ++sub) {
+      for (int sub = 0; sub < C::EPI_COLS / C::EPI_SUB; ++sub) {
         if (lane == 0) bulk_wait_group_read<0>();  // the staging sub-tile is free again
         __syncwarp();
-        // 8 groups of 8 columns: alpha * acc + bias, bf16, one 16-byte store each
-        // into a 32 x 64 staging sub-tile (128 B rows, 128-byte swizzle)
+        // groups of 8 columns: alpha * acc + bias, bf16, one 16-byte store each
+        // into the 32 x EPI_SUB staging sub-tile (64 B rows, 64-byte swizzle:
+        // 16-byte chunk c of row l sits at chunk c ^ ((l / 2) % 4))
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int grp = h * (C::EPI_COLS / 8) + sub * 8 + j;  // 8-column group within the tile
+        for (int j = 0; j < C::EPI_SUB / 8; ++j) {
+          const int grp = h * (C::EPI_COLS / 8) + sub * (C::EPI_SUB / 8) + j;  // 8-column group in the tile
           uint32_t bw[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) bw[e] = __shfl_sync(0xffffffffu, bias_l[e], grp);
           uint32_t pk[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int c = sub * 64 + j * 8 + 2 * e;
+            const int c = sub * C::EPI_SUB + j * 8 + 2 * e;
             float v0 = __uint_as_float(r[c]), v1 = __uint_as_float(r[c + 1]);
             if constexpr (F == Fmt::NVFP4) { v0 *= alpha; v1 *= alpha; }
             v0 += __uint_as_float(bw[e] << 16);
@@ -450,14 +476,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
             const __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
             pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
           }
-          const uint32_t addr = stage_buf + lane * 128 + ((j ^ (lane & 7)) << 4);
+          static_assert(C::EPI_SUB == 32, "staging swizzle");
+          const uint32_t addr = stage_buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]),
                        "r"(pk[2]), "r"(pk[3])
                        : "memory");
         }
         fence_proxy_async_smem();
         __syncwarp();
-        const int x = col_w + sub * 64;
+        const int x = col_w + sub * C::EPI_SUB;
         if (lane == 0 && row0 < M && x < N) {
           tma_store_2d(&tmap_y, stage_buf, x, row0);
           bulk_commit_group();
