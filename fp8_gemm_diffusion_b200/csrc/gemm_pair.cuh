@@ -15,14 +15,17 @@
 //               barrier (cta_group::2 loads, no multicast).
 //   warp 1      tensor memory (cta_group::2 allocation); on the even CTA one
 //               lane issues the MMAs and commits to both CTAs' barriers
-//               (multicast commit): A/B stage free (the scale set that the
-//               stage read is free from then on too) and accumulator full.
+//               (multicast commit): stage free (its A/B slot and its scale
+//               set) and accumulator full.  A stage's commit is issued after
+//               the next stage's wait, so the wait never follows a commit.
 //   warp 2      scale loader: the scale chunks of each stage (A's 128 rows and
 //               all BN columns of B: each CTA's tensor memory needs B's) into
 //               a separate ring that runs ahead of the A/B ring.
 //   warps 4-7   scale writers, one per tensor-memory sub-partition: chunk rows
-//               from shared memory into one of NS sets of tensor-memory
-//               columns with tcgen05.st, so no tcgen05.cp sits between MMAs.
+//               from shared memory into the stage's set of tensor-memory
+//               columns with tcgen05.st, so no tcgen05.cp sits between MMAs;
+//               they arrive on the even CTA's full barrier of the stage, which
+//               thus completes when A, B and all scales are in place.
 //   warps 8-15  epilogue, sub-partition warp % 4, column half (warp / 4) % 2:
 //               the warp's accumulator columns into registers, release of the
 //               accumulator, then alpha, bias, bf16, 64-byte swizzled staging
@@ -65,14 +68,12 @@ struct PairCfg {
   static constexpr uint32_t SF_TX = SFA_BYTES + SFB_BYTES;  // this CTA's scales
   static constexpr int SF_SLOT_BYTES = SCALED ? (SFA_BYTES + SFB_BYTES + 1023) / 1024 * 1024 : 0;
   static constexpr int SF_SLOTS = SCALED ? (F == Fmt::NVFP4 ? 4 : 8) : 0;
-  // tensor memory: the accumulator (BN columns), then NS scale sets (A chunks,
-  // then B chunks in MMA-major order, 4 columns each)
+  // tensor memory: the accumulator (BN columns), then one scale set per A/B
+  // stage (A chunks, then B chunks in MMA-major order, 4 columns each)
   static constexpr int SF_SET_COLS = (SF_CHUNKS + NRB * SF_CHUNKS) * 4;
   static constexpr int SF_COL = BN;
   static constexpr int SFB_OFF = SF_CHUNKS * 4;
   static constexpr int TMEM_COLS = 512;
-  // scale sets in tensor memory: stage k uses set k % NS, free again when the
-  // MMAs of stage k - NS have completed (that stage's A/B commit)
   static constexpr int NS_FIT = SCALED ? (TMEM_COLS - BN) / SF_SET_COLS : 64;
   // warp roles, one warpgroup each for (producer, MMA, scale loader, spare),
   // the scale writers and the two halves of the epilogue
@@ -88,8 +89,11 @@ struct PairCfg {
   static constexpr int BAR_BYTES = 512;
   static constexpr int STAGES_FIT =
       (232448 - 1024 - BAR_BYTES - EPI_BYTES - SF_SLOTS * SF_SLOT_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr int NS = NS_FIT < STAGES ? NS_FIT : STAGES;
+  static constexpr int STAGES_MIN = STAGES_FIT < NS_FIT ? STAGES_FIT : NS_FIT;
+  static constexpr int STAGES = STAGES_MIN > 8 ? 8 : STAGES_MIN;
+  // arrivals that complete a stage's full barrier besides the A/B bytes: the
+  // producer's expect-tx and the scale writers of both CTAs
+  static constexpr int FULL_ARRIVALS = 1 + (SCALED ? 2 * SF_WARPS : 0);
   static_assert(STAGES >= 2, "shared / tensor memory");
   static constexpr int SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + EPI_BYTES + BAR_BYTES;
@@ -140,7 +144,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
                      const __grid_constant__ CUtensorMap tmap_sfb,
                      const __grid_constant__ CUtensorMap tmap_y, const PairArgs args) {
   using C = PairCfg<F, BN>;
-  constexpr int S = C::STAGES, R = C::SF_SLOTS, NS = C::NS;
+  constexpr int S = C::STAGES, R = C::SF_SLOTS;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -148,13 +152,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
   const uint32_t sf_base = base + S * C::STAGE_BYTES;
   const uint32_t epi_base = sf_base + R * C::SF_SLOT_BYTES;
   const uint32_t bar_base = epi_base + C::EPI_BYTES;
-  // barriers: [full S][empty S][sf_full R][sf_empty R][sf_ready S][tfull][tempty][drain]
-  auto full_bar = [&](int s) { return bar_base + 8u * s; };                 // even CTA: A/B landed
+  // barriers: [full S][empty S][sf_full R][sf_empty R][tfull][tempty][drain]
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };  // even CTA: A/B landed, scales written
   auto empty_bar = [&](int s) { return bar_base + 8u * (S + s); };          // both: A/B stage free
   auto sf_full_bar = [&](int r) { return bar_base + 8u * (2 * S + r); };    // both: own scales landed
   auto sf_empty_bar = [&](int r) { return bar_base + 8u * (2 * S + R + r); };  // both: slot read
-  auto sf_ready_bar = [&](int n) { return bar_base + 8u * (2 * S + 2 * R + n); };  // even: set written
-  const uint32_t tfull_bar = bar_base + 8u * (2 * S + 2 * R + NS);
+  const uint32_t tfull_bar = bar_base + 8u * (2 * S + 2 * R);
   const uint32_t tempty_bar = tfull_bar + 8u;
   const uint32_t drain_bar = tfull_bar + 16u;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + (tfull_bar + 24u - base));
@@ -177,14 +180,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(full_bar(s), 1);
+      mbar_init(full_bar(s), C::FULL_ARRIVALS);
       mbar_init(empty_bar(s), 1);
     }
     for (int r = 0; r < R; ++r) {
       mbar_init(sf_full_bar(r), 1);
       mbar_init(sf_empty_bar(r), C::SF_WARPS);
     }
-    for (int n = 0; n < NS; ++n) mbar_init(sf_ready_bar(n), 2 * C::SF_WARPS);
     mbar_init(tfull_bar, 1);
     mbar_init(tempty_bar, 2 * C::EPI_WARPS);
     mbar_init(drain_bar, 1);
@@ -243,7 +245,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         // let every armed stage land before the pair can exit
         for (int i = 0; i < S && i < issued; ++i) {
           if (--s < 0) { s = S - 1; ph ^= 1u; }
-          mbar_wait_bounded(full_bar(s), ph);
+          if (!mbar_wait_bounded(full_bar(s), ph)) break;
         }
       }
     }
@@ -251,8 +253,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
     // ------------------------------------------------------------ MMA issuer
     // (one thread: keep the per-stage work to a few instructions)
     if (lane == 0 && rank == 0) {
-      int s = 0, n = 0;
-      uint32_t ph = 0, nph = 0, acc_ph = 0;
+      int s = 0, pend = -1;  // pend: stage whose MMAs are issued but not committed
+      uint32_t ph = 0, acc_ph = 0;
       bool ok = true;
       const uint64_t adesc0 = desc_kmajor_sw128(base);
       const uint64_t bdesc0 = desc_kmajor_sw128(base + C::A_BYTES);
@@ -268,10 +270,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         tc_fence_after();
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(full_bar(s), ph)) { ok = false; break; }
-          if (C::SCALED && !mbar_wait_bounded(sf_ready_bar(n), nph)) { ok = false; break; }
+          // the previous stage's commit: after this wait, since a barrier wait
+          // issued right behind a commit takes a few hundred cycles longer
+          if (pend >= 0) tc_commit_pair(empty_bar(pend));
           tc_fence_after();
           const uint64_t adesc = adesc0 + DSTEP * s, bdesc = bdesc0 + DSTEP * s;
-          const uint32_t sf = tmem_base + C::SF_COL + n * C::SF_SET_COLS;
+          const uint32_t sf = tmem_base + C::SF_COL + s * C::SF_SET_COLS;
           int nmma = C::MMAS;
           if constexpr (F == Fmt::NVFP4) {
             if (kb == num_kb - 1) nmma = K / 64 - kb * C::MMAS;  // K % 256 != 0: partial last stage
@@ -294,10 +298,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
               }
             }
           }
-          tc_commit_pair(empty_bar(s));  // frees A/B stage s (and scale set n, NS stages on)
+          pend = s;  // committed (A/B slot and scale set s free) after the next wait
           if (++s == S) { s = 0; ph ^= 1u; }
-          if (++n == NS) { n = 0; nph ^= 1u; }
         }
+        if (pend >= 0) tc_commit_pair(empty_bar(pend));
+        pend = -1;
         if (!ok) break;
         tc_commit_pair(tfull_bar);
       }
@@ -352,10 +357,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
     // every sub-partition, column r / 32 of the chunk's four).
     if constexpr (C::SCALED) {
       const uint32_t q = static_cast<uint32_t>(warp & 3);
-      const uint32_t leader_ready0 = map_to_cta(sf_ready_bar(0), 0);
+      const uint32_t leader_full0 = map_to_cta(full_bar(0), 0);
       constexpr int NCH = C::SF_CHUNKS * (1 + C::NRB);  // A chunks, then B chunks
-      int r = 0, n = 0, js = 0;
-      uint32_t rph = 0, jph = 0;
+      int r = 0, n = 0;
+      uint32_t rph = 0, nph = 0;
       for (int g = 0; g < total_kb; ++g) {
         if (!mbar_wait_bounded(sf_full_bar(r), rph)) break;
         const uint32_t slot = sf_base + r * C::SF_SLOT_BYTES;
@@ -376,12 +381,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(sf_empty_bar(r));  // slot read: the loader may refill it
-        // set n is free once the MMAs of stage j = g - NS (A/B slot js, that
-        // slot's completion number j / S) have completed
-        if (g >= NS) {
-          if (!mbar_wait_bounded(empty_bar(js), jph)) break;
-          if (++js == S) { js = 0; jph ^= 1u; }
-        }
+        // set n is free once the MMAs of stage g - S have completed; the full
+        // barrier of that stage has completed too, so the arrival below counts
+        // towards stage g
+        if (g >= S && !mbar_wait_bounded(empty_bar(n), nph ^ 1u)) break;
         tc_fence_after();
         const uint32_t t = tmem_base + (q * 32u << 16) + C::SF_COL + n * C::SF_SET_COLS;
         if constexpr (NCH * 4 % 16 == 0) {
@@ -400,9 +403,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(leader_ready0 + 8u * n);
+        if (lane == 0) mbar_arrive_remote(leader_full0 + 8u * n);
         if (++r == R) { r = 0; rph ^= 1u; }
-        if (++n == NS) n = 0;
+        if (++n == S) { n = 0; nph ^= 1u; }
       }
     }
   } else {
