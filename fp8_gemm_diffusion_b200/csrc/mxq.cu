@@ -186,6 +186,71 @@ mxq_status launch_quant_nvfp4(const void* x, int64_t rows, int64_t k, int64_t ld
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
+// ---- single-pass NVFP4 quantisation (rows held in shared memory)
+constexpr int kFusedMaxGrid = 256;          // tag capacity in the workspace header
+constexpr size_t kFusedSmemLimit = 227 * 1024 - 1024;  // dynamic bytes, static ones kept aside
+
+struct FusedPlan {
+  int grid = 0, rows_per_cta = 0;
+  size_t smem = 0;
+};
+
+// One CTA per SM, each holding ceil(rows / SMs) rows and one mbarrier per row.
+FusedPlan plan_fused(int64_t rows, int64_t k, int sms) {
+  FusedPlan p;
+  if (rows <= 0 || k <= 0 || sms <= 0) return p;
+  const int64_t rpc = (rows + sms - 1) / sms;
+  const size_t smem = static_cast<size_t>(rpc) * static_cast<size_t>(k) * 2 + 8 * static_cast<size_t>(rpc);
+  const int64_t grid = (rows + rpc - 1) / rpc;
+  if (smem > kFusedSmemLimit || grid > kFusedMaxGrid) return p;
+  p.grid = static_cast<int>(grid);
+  p.rows_per_cta = static_cast<int>(rpc);
+  p.smem = smem;
+  return p;
+}
+
+// Cooperative launch (the grid barrier needs every CTA resident), with
+// programmatic stream serialization when the driver accepts both.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_coop(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                        Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e == cudaSuccess) return e;
+  cudaGetLastError();
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+mxq_status launch_quant_nvfp4_fused(const void* x, int64_t rows, int64_t k, int64_t ld,
+                                    const FusedPlan& p, mxq::FusedSync* sync, uint8_t* codes,
+                                    uint8_t* sf, float* g, float* amax_out, cudaStream_t s,
+                                    int dev) {
+  constexpr uint32_t bit = 1u << 20;  // GEMM instantiations use the low bits
+  if (!(g_dev[dev].smem_attr_set.load(std::memory_order_acquire) & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(mxq::quantize_nvfp4_fused_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kFusedSmemLimit));
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_dev[dev].smem_attr_set.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  cudaError_t e = launch_coop(mxq::quantize_nvfp4_fused_kernel, dim3(p.grid), dim3(mxq::kFusedThreads),
+                              p.smem, s, static_cast<const __nv_bfloat16*>(x), static_cast<int>(rows),
+                              static_cast<int>(k), ld, p.rows_per_cta, sync, codes, sf, g, amax_out);
+  return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
+}
+
 mxq_status launch_quant_mxfp8(const void* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
                               uint8_t* sf, cudaStream_t s, int sms) {
   cudaError_t e = launch_pdl(mxq::quantize_mxfp8_kernel, dim3(quant_grid(rows, sms)),
@@ -357,10 +422,15 @@ bool valid_format(int f) { return f == MXQ_NVFP4 || f == MXQ_MXFP8 || f == MXQ_B
 
 // Byte layout of the weight storage and of the activation workspace:
 // [0,4) amax, [4,8) g, then (workspace only) the per-block amax partials at
-// [256, 256 + 4 * kMaxAmaxPartials), then the codes and the scales, each
-// 256-byte aligned.
+// [256, 256 + 4 * kMaxAmaxPartials), the single-pass quantiser's barrier
+// state (mxq::FusedSync, 256 bytes, then 8 bytes per CTA) from 4352, then
+// the codes and the scales, each 256-byte aligned.
 constexpr size_t kPartialsOff = 256;
-constexpr size_t kWorkspaceHeader = 8192;  // holds the partials
+constexpr size_t kSyncOff = 4352;
+constexpr size_t kWorkspaceHeader = 8192;
+static_assert(kPartialsOff + 4 * mxq::kMaxAmaxPartials <= kSyncOff, "workspace header");
+static_assert(kSyncOff + sizeof(mxq::FusedSync) + 8 * kFusedMaxGrid <= kWorkspaceHeader,
+              "workspace header");
 struct QuantLayout {
   size_t codes_off, sf_off, total;
 };
@@ -590,11 +660,21 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
   uint8_t* sf = base + l.sf_off;
   if (f == MXQ_NVFP4) {
     float* partials = reinterpret_cast<float*>(base + kPartialsOff);
-    int n_partials = 0;
-    if ((st = launch_amax_partials(x_bf16, M, K, K, partials, &n_partials, s, sms)) != MXQ_OK) return st;
-    if ((st = launch_quant_nvfp4(x_bf16, M, K, K, partials, n_partials, codes, sf, g, amax, s, sms)) !=
-        MXQ_OK)
-      return st;
+    const FusedPlan plan = plan_fused(M, K, sms);
+    if (plan.grid > 0) {
+      // the activation fits in shared memory: one pass over HBM
+      st = launch_quant_nvfp4_fused(x_bf16, M, K, K, plan,
+                                    reinterpret_cast<mxq::FusedSync*>(base + kSyncOff), codes, sf,
+                                    g, amax, s, dev);
+      if (st != MXQ_OK) return st;
+    } else {
+      int n_partials = 0;
+      if ((st = launch_amax_partials(x_bf16, M, K, K, partials, &n_partials, s, sms)) != MXQ_OK)
+        return st;
+      if ((st = launch_quant_nvfp4(x_bf16, M, K, K, partials, n_partials, codes, sf, g, amax, s,
+                                   sms)) != MXQ_OK)
+        return st;
+    }
   } else {
     if ((st = launch_quant_mxfp8(x_bf16, M, K, K, codes, sf, s, sms)) != MXQ_OK) return st;
   }

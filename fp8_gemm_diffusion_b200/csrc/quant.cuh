@@ -3,6 +3,8 @@
 //   amax_kernel           max |x| of a bf16 matrix -> one fp32 (atomicMax on
 //                         the bit pattern, valid because |x| >= 0)
 //   quantize_nvfp4_kernel per 16-element block: E4M3 scale, E2M1 codes
+//   quantize_nvfp4_fused_kernel  both of the above in one pass, for an
+//                         activation that fits in the grid's shared memory
 //   quantize_mxfp8_kernel per 32-element block: E8M0 scale, E4M3 codes
 //
 // Source: B200 MXFP8/NVFP4 diffusion article, Glossary "Microscaling
@@ -202,6 +204,21 @@ __device__ __forceinline__ void zero_sf_padding(uint8_t* __restrict__ sf, int ro
   }
 }
 
+// One 16-byte vector (8 elements) of a row: lanes 2i and 2i+1 of the warp
+// hold the two halves of one 16-element block (every lane must call this).
+// Returns the 8 E2M1 codes packed; sfc receives the block's E4M3 scale code.
+__device__ __forceinline__ uint32_t nvfp4_vector(float (&f)[8], float g, float six_g,
+                                                 uint32_t& sfc) {
+  float bmax = absmax8(f);
+  bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));  // 16-element block
+  sfc = cvt_e4m3x2(bmax / six_g, 0.0f) & 0xFFu;
+  const float s = e4m3_value(sfc) * g;
+  const float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = f[i] * inv;
+  return cvt_e2m1x8(f);
+}
+
 // amax_in: n_amax values whose max is the tensor's amax (1 value, or the
 // per-block partials of amax_kernel).
 __global__ void __launch_bounds__(kQuantThreads)
@@ -240,19 +257,232 @@ __global__ void __launch_bounds__(kQuantThreads)
         if (v - lane >= vpr) break;  // warp-uniform
         float f[8];
         bf16x8_to_f32(u[j], f);
-        float bmax = absmax8(f);
-        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));  // 16-element block
-        const uint32_t sfc = cvt_e4m3x2(bmax / six_g, 0.0f) & 0xFFu;
-        const float s = e4m3_value(sfc) * g;
-        const float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = f[i] * inv;
-        const uint32_t packed = cvt_e2m1x8(f);
+        uint32_t sfc;
+        const uint32_t packed = nvfp4_vector(f, g, six_g, sfc);
         if (v < vpr) {
           crow[v] = packed;
           if ((v & 1) == 0) sf[sf_offset(r, v >> 1, c4)] = static_cast<uint8_t>(sfc);
         }
       }
+    }
+  }
+  zero_sf_padding(sf, rows, k >> 4);
+}
+
+// ------------------------------------------------ NVFP4 in a single pass
+// For an activation that fits in the grid's shared memory.  Each CTA copies
+// its rows into shared memory once (bulk copies, one mbarrier per row), takes
+// their maximum, the CTAs exchange maxima through a grid-wide barrier, and
+// each CTA quantises its rows from shared memory: the activation crosses HBM
+// once instead of twice, and one launch replaces two.
+//
+// Grid barrier, state in caller memory with any initial contents
+// (FusedSync below, then tags[grid]).  Every exchanged word is 64 bits,
+// written and read whole (single-copy atomic), so no fences are needed:
+//   key     (epoch & 0xffff) << 48 | (~epoch & 0xffff) << 32, where epoch is
+//           read by every CTA at entry and advanced by CTA 0 once all CTAs
+//           have arrived (so no CTA reads the advanced value in the same
+//           launch).  Zeroed or byte-filled memory never matches a key (its
+//           two halves are not complements);
+//   tags[b] key | bits(maximum of CTA b), its arrival;
+//   done    key | bits(amax): CTA 0 waits for every tag, publishes done and
+//           clears the tags; every CTA waits on that one word, so the polling
+//           stays off the tag lines.
+// The launch is cooperative (all CTAs resident together) and every wait is
+// bounded: on timeout the CTA records kErrTimeout and leaves its rows
+// unquantised (CTA 0 still advances the epoch, so a later launch never
+// matches a word of this one).
+constexpr int kFusedThreads = 1024;
+constexpr int kFusedWarps = kFusedThreads / 32;
+
+struct FusedSync {                 // 256 bytes, then tags[grid]
+  unsigned int epoch;
+  unsigned int pad0;
+  unsigned long long done;
+  unsigned int pad1[60];
+};
+static_assert(sizeof(FusedSync) == 256, "FusedSync layout");
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Relaxed loads: independent, so a lane keeps several in flight at once.
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned int ld_relaxed_u32(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(addr));
+  return r;
+}
+
+// One 16-element block held by one lane: the same arithmetic as
+// nvfp4_vector, with the block-level steps done once per block.  Returns the
+// 16 E2M1 codes (element 2i in the low nibble of byte i); sfc receives the
+// block's E4M3 scale code.
+__device__ __forceinline__ uint2 nvfp4_block16(float (&f)[16], float g, float six_g,
+                                               uint32_t& sfc) {
+  float bmax = fabsf(f[0]);
+#pragma unroll
+  for (int i = 1; i < 16; ++i) bmax = fmaxf(bmax, fabsf(f[i]));
+  sfc = cvt_e4m3x2(bmax / six_g, 0.0f) & 0xFFu;
+  const float s = e4m3_value(sfc) * g;
+  const float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
+  float lo[8], hi[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    lo[i] = f[i] * inv;
+    hi[i] = f[8 + i] * inv;
+  }
+  return make_uint2(cvt_e2m1x8(lo), cvt_e2m1x8(hi));
+}
+
+constexpr unsigned long long kKeyMask = 0xFFFFFFFF00000000ull;
+
+// Bounded spin until the word's upper half equals `key`; its lower half out.
+__device__ __forceinline__ bool spin_for_key(const unsigned long long* p, unsigned long long key,
+                                             uint32_t& value) {
+  const uint64_t t0 = globaltimer_ns();
+  unsigned long long w;
+  while (((w = ld_relaxed_u64(p)) & kKeyMask) != key) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+  value = static_cast<uint32_t>(w);
+  return true;
+}
+
+// Dynamic shared memory: rows_per_cta rows of k bf16, then one mbarrier per row.
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    quantize_nvfp4_fused_kernel(const __nv_bfloat16* __restrict__ x, int rows, int k, int64_t ld,
+                                int rows_per_cta, FusedSync* sync, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                float* __restrict__ g_out, float* __restrict__ amax_out) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float s_red[kFusedWarps];
+  __shared__ float s_amax;
+  __shared__ unsigned int s_epoch;
+  __shared__ int s_ok;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t row_bytes = static_cast<uint32_t>(k) * 2u;
+  const uint32_t rows_s = smem_u32(smem);
+  const uint32_t bar0 = rows_s + static_cast<uint32_t>(rows_per_cta) * row_bytes;
+  const int r0 = blockIdx.x * rows_per_cta;
+  const int nr = min(rows_per_cta, rows - r0);
+  const int vpr = k >> 3;  // 16-byte vectors per row
+  unsigned long long* const tags = reinterpret_cast<unsigned long long*>(sync + 1);
+
+  grid_dep_wait();  // x is the previous kernel's output
+  if (threadIdx.x == 0) {
+    s_epoch = ld_relaxed_u32(&sync->epoch);
+    for (int i = 0; i < nr; ++i) mbar_init(bar0 + 8u * i, 1);
+    fence_barrier_init();
+    for (int i = 0; i < nr; ++i) {
+      mbar_arrive_expect_tx(bar0 + 8u * i, row_bytes);
+      bulk_load(rows_s + static_cast<uint32_t>(i) * row_bytes, x + static_cast<int64_t>(r0 + i) * ld,
+                row_bytes, bar0 + 8u * i);
+    }
+  }
+  __syncthreads();
+  grid_dep_launch();
+
+  // ---- this CTA's maximum, row by row as the rows land
+  float m = 0.0f;
+  for (int i = warp; i < nr; i += kFusedWarps) {
+    mbar_wait_bounded(bar0 + 8u * i, 0);
+    const uint32_t row = rows_s + static_cast<uint32_t>(i) * row_bytes;
+    for (int v = lane; v < vpr; v += 32) {
+      float f[8];
+      bf16x8_to_f32(lds_v4(row + 16u * v), f);
+      m = fmaxf(m, absmax8(f));
+    }
+  }
+  m = warp_max(m);
+  if (lane == 0) s_red[warp] = m;
+  __syncthreads();
+
+  // ---- grid barrier: arrive, CTA 0 gathers and publishes, everyone reads
+  const uint32_t e16 = s_epoch & 0xFFFFu;
+  const unsigned long long key =
+      (static_cast<unsigned long long>(e16) << 48) | (static_cast<unsigned long long>(~e16 & 0xFFFFu) << 32);
+  if (warp == 0) {
+    float b = lane < kFusedWarps ? s_red[lane] : 0.0f;
+    b = warp_max(b);
+    if (lane == 0) st_relaxed_u64(tags + blockIdx.x, key | __float_as_uint(b));
+    __syncwarp();
+    bool ok = true;
+    if (blockIdx.x == 0) {
+      const int nb = gridDim.x;
+      const uint64_t t0 = globaltimer_ns();
+      float a = 0.0f;
+      while (true) {
+        bool mine = true;
+        a = 0.0f;
+        for (int c = lane; c < nb; c += 32) {
+          const unsigned long long w = ld_relaxed_u64(tags + c);
+          mine &= (w & kKeyMask) == key;
+          a = fmaxf(a, __uint_as_float(static_cast<uint32_t>(w)));
+        }
+        if (__all_sync(0xffffffffu, mine)) break;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          ok = false;
+          break;
+        }
+      }
+      a = warp_max(a);
+      if (ok && lane == 0) st_relaxed_u64(&sync->done, key | __float_as_uint(a));
+      for (int c = lane; c < nb; c += 32) st_relaxed_u64(tags + c, 0ull);
+      if (lane == 0) sync->epoch = s_epoch + 1u;  // every CTA read the epoch before its tag
+    }
+    if (lane == 0) {
+      uint32_t bits = 0;
+      ok = ok && spin_for_key(&sync->done, key, bits);
+      if (ok) s_amax = __uint_as_float(bits);
+      else record_error(kErrTimeout);
+      s_ok = ok ? 1 : 0;
+    }
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  const float a = s_amax;
+  const float g = nvfp4_global_scale(a);
+  const float six_g = 6.0f * g;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *g_out = g;
+    if (amax_out != nullptr) *amax_out = a;
+  }
+
+  // ---- quantise this CTA's rows from shared memory: one lane per 16-element block
+  const int bpr = k >> 4;       // blocks per row
+  const uint32_t c4 = static_cast<uint32_t>(k >> 6);
+  for (int i = warp; i < nr; i += kFusedWarps) {
+    const int r = r0 + i;
+    const uint32_t row = rows_s + static_cast<uint32_t>(i) * row_bytes;
+    uint2* crow = reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * (k >> 1));
+    // this row's scale bytes: 512-byte tile (r / 128, c / 4), byte (r % 32) * 16 + (r / 32 % 4) * 4 + c % 4
+    uint8_t* sf_row = sf + static_cast<int64_t>(r >> 7) * c4 * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
+    for (int c = lane; c < bpr; c += 32) {
+      const uint4 u0 = lds_v4(row + 32u * c), u1 = lds_v4(row + 32u * c + 16u);
+      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      float f[16];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        f[2 * j] = __uint_as_float(w[j] << 16);
+        f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+      uint32_t sfc;
+      crow[c] = nvfp4_block16(f, g, six_g, sfc);
+      sf_row[(c >> 2) * 512 + (c & 3)] = static_cast<uint8_t>(sfc);
     }
   }
   zero_sf_padding(sf, rows, k >> 4);
