@@ -202,7 +202,9 @@ def run_gpu(args, rank, world, local_rank):
                              h.codes, h.sf, h.g_dev if fmt == "nvfp4" else None, bias, st["y"],
                              stream=stream)
 
-    launches_per_step = 3 if fmt == "nvfp4" else 2  # (amax,) quantise, GEMM
+    # kernels one mxq_linear call launches here (the library's own dispatch decision)
+    launches_per_step = mxq.linear_kernel_count(base_w.handle, M)
+    assert launches_per_step > 0, launches_per_step
     dist = world > 1
     if dist:
         import torch.distributed as tdist

@@ -95,6 +95,8 @@ _linear = _proto("mxq_linear", _int, ctypes.POINTER(mxq_weight), _ptr, _i64, _pt
                  ctypes.POINTER(mxq_linear_opts), _ptr)
 _linear_noalloc = _proto("mxq_linear_noalloc", _int, ctypes.POINTER(mxq_weight), _ptr, _i64,
                          _ptr, ctypes.POINTER(mxq_linear_opts), _ptr)
+_linear_kernel_count = _proto("mxq_linear_kernel_count", _int, ctypes.POINTER(mxq_weight), _i64,
+                              ctypes.POINTER(mxq_linear_opts))
 _get_device_error = _proto("mxq_get_device_error", _int, _ptr)
 _convert_f32 = _proto("mxq_convert_f32", _int, _ptr, _i64, _int, _ptr, _ptr)
 
@@ -104,7 +106,7 @@ EXPORTED = [
     "mxq_codes_bytes", "mxq_amax", "mxq_quantize_nvfp4", "mxq_quantize_mxfp8",
     "mxq_gemm_blockscaled", "mxq_weight_storage_bytes", "mxq_weight_prepare",
     "mxq_linear_path", "mxq_linear_workspace_bytes", "mxq_linear", "mxq_get_device_error",
-    "mxq_convert_f32", "mxq_linear_noalloc",
+    "mxq_convert_f32", "mxq_linear_noalloc", "mxq_linear_kernel_count",
 ]
 
 #: Capacity of the static device scratch of mxq_linear_noalloc (MXQ_NOALLOC_SCRATCH_BYTES).
@@ -225,6 +227,11 @@ def _opts(min_dim):
 
 def linear_path(w: mxq_weight, M: int, min_dim=None) -> int:
     return _linear_path(ctypes.byref(w), M, _opts(min_dim))
+
+
+def linear_kernel_count(w: mxq_weight, M: int, min_dim=None) -> int:
+    """Kernels one mxq_linear call launches for these arguments (-1: no device)."""
+    return _linear_kernel_count(ctypes.byref(w), M, _opts(min_dim))
 
 
 def linear_workspace_bytes(M: int, K: int, fmt) -> int:

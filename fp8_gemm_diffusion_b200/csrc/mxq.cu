@@ -683,6 +683,16 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
                      y_bf16, N, s);
 }
 
+int mxq_linear_kernel_count(const mxq_weight* w, int64_t M, const mxq_linear_opts* opts) {
+  if (w == nullptr || M <= 0 || w->N <= 0) return 0;
+  const int path = mxq_linear_path(w, M, opts);
+  if (path == MXQ_BF16) return 1;
+  if (path == MXQ_MXFP8) return 2;
+  int dev, sms;
+  if (current_device(&dev, &sms) != MXQ_OK) return -1;
+  return plan_fused(M, w->K, sms).grid > 0 ? 2 : 3;
+}
+
 mxq_status mxq_get_device_error(mxq_stream_t stream) {
   int dev, sms;
   mxq_status st = current_device(&dev, &sms);

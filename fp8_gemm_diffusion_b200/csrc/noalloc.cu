@@ -18,10 +18,10 @@
 //     array's device address with cudaGetSymbolAddress and caches it; make
 //     that first call before any stream capture.
 //   * All calls on a device share the one array and it keeps the previous
-//     call's contents.  The amax slot, the only value that must start at
-//     zero, is cleared on the stream by every call before it is used; codes
-//     and scales are fully rewritten.  Calls whose work can overlap on the
-//     GPU (different streams, or several host threads without ordering)
+//     call's contents.  mxq_linear needs no value of its workspace to start
+//     at zero: codes and scales are fully rewritten and the quantiser's amax
+//     exchange is valid from any contents.  Calls whose work can overlap on
+//     the GPU (different streams, or several host threads without ordering)
 //     race on the array: serialise them, e.g. on one stream.
 #include <cuda_runtime.h>
 

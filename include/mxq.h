@@ -213,7 +213,13 @@ size_t mxq_linear_workspace_bytes(int64_t M, int64_t K, mxq_format f);
  * amax -> NVFP4 quantise -> block-scaled GEMM, or MXFP8 quantise ->
  * block-scaled GEMM.  ws: device workspace of at least
  * mxq_linear_workspace_bytes(M, K, w->format) bytes, 256-byte aligned
- * (unused on the bf16 path; may be NULL there).
+ * (unused on the bf16 path; may be NULL there).  Its contents on entry do not
+ * matter (nothing in it has to start at zero).
+ * NVFP4 activations that fit in the shared memory of one CTA per SM are
+ * quantised by one cooperative kernel (amax and quantisation in one pass
+ * over HBM, the amax exchanged through a bounded grid barrier whose state
+ * lives in the workspace); larger ones by two kernels (partial maxima, then
+ * quantisation).  Calls sharing one workspace must be ordered on the GPU.
  */
 mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* y_bf16,
                       void* ws, size_t ws_bytes, const mxq_linear_opts* opts,
@@ -236,10 +242,10 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
  *  - The first call on a device (with that device current) looks up the
  *    array's address and caches it; make that first call before any stream
  *    capture.
- *  - All calls share the array and it keeps the previous call's contents; the
- *    one value that must start at zero (the activation amax) is cleared on the
- *    stream by every call.  Calls that can overlap on the GPU (other streams,
- *    unordered host threads) race on the array: serialise them.
+ *  - All calls share the array and it keeps the previous call's contents,
+ *    which is all mxq_linear needs (no value in its workspace has to start at
+ *    zero).  Calls that can overlap on the GPU (other streams, unordered host
+ *    threads) race on the array: serialise them.
  *  - A quantised path whose workspace (mxq_linear_workspace_bytes) exceeds
  *    MXQ_NOALLOC_SCRATCH_BYTES returns MXQ_ERR_WORKSPACE and enqueues nothing;
  *    the bf16 path needs no workspace.
@@ -248,6 +254,16 @@ mxq_status mxq_linear_noalloc(const mxq_weight* w, const void* x_bf16, int64_t M
                               const mxq_linear_opts* opts, mxq_stream_t stream);
 
 /* ---------------------------------------------------- diagnostics ------- */
+
+/*
+ * mxq_linear_kernel_count - how many kernels one mxq_linear call with these
+ * arguments launches on the current device: 1 (bf16 GEMM), 2 (MXFP8
+ * quantise + GEMM, or single-pass NVFP4 quantise + GEMM) or 3 (NVFP4 partial
+ * maxima + quantise + GEMM); 0 when M or N is 0 (nothing is launched) or w
+ * is NULL; -1 when the current device cannot be queried.  Uses the same
+ * decisions as mxq_linear.  No GPU work.
+ */
+int mxq_linear_kernel_count(const mxq_weight* w, int64_t M, const mxq_linear_opts* opts);
 
 /*
  * mxq_get_device_error - synchronise `stream`, then read and clear the

@@ -131,3 +131,16 @@ def test_linear_path_follows_selection_rule():
     assert mxq.linear_path(w, 1024, min_dim=2048) == mxq.BF16
     w.keep_bf16 = 1
     assert mxq.linear_path(w, 8192) == mxq.BF16
+
+
+def test_linear_kernel_count_host_cases():
+    w = mxq.mxq_weight(format=mxq.MXFP8, keep_bf16=0, N=1024, K=1024)
+    assert mxq.linear_kernel_count(w, 0) == 0            # nothing launched
+    assert mxq.linear_kernel_count(w, 1023) == 1         # bf16 GEMM
+    assert mxq.linear_kernel_count(w, 1024) == 2         # MXFP8 quantise + GEMM
+    w = mxq.mxq_weight(format=mxq.NVFP4, keep_bf16=0, N=0, K=1024)
+    assert mxq.linear_kernel_count(w, 4096) == 0
+    if not torch.cuda.is_available():
+        # the NVFP4 choice (one or two quantiser kernels) depends on the SM count
+        w = mxq.mxq_weight(format=mxq.NVFP4, keep_bf16=0, N=1024, K=1024)
+        assert mxq.linear_kernel_count(w, 4096) == -1

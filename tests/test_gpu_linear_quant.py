@@ -125,3 +125,10 @@ def test_single_pass_wide_dynamic_range():
     ws = _run(_weight(K), A, 0xFF)
     _check(ws, A)
     assert mxq.get_device_error() == mxq.OK
+
+
+def test_kernel_count_matches_the_path_taken():
+    w = _weight(3072)
+    assert mxq.linear_kernel_count(w.handle, 4608, min_dim=1) == 2   # single pass + GEMM
+    w = _weight(4096)
+    assert mxq.linear_kernel_count(w.handle, 4608, min_dim=1) == 3   # amax + quantise + GEMM
