@@ -351,33 +351,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
   } else if (warp < C::EPI_WARP0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_SFW));
     // ------------------------------------------------ scale factors -> TMEM
-    // Each warp writes the 32 lanes of its sub-partition: lane l receives row l
-    // of every 512-byte scale chunk of the stage (16 bytes = 4 columns), the
-    // layout the block-scaled MMA reads (row r's scales in lane r % 32 of
-    // every sub-partition, column r / 32 of the chunk's four).
+    // Each warp writes the 32 lanes of its sub-partition q.  A 512-byte chunk
+    // row l holds four 4-byte words, word m = the scales of row l + 32 m.
+    // B's chunks go to every sub-partition whole (4 columns: every lane of D
+    // needs every column's scales).  A's chunks need only their diagonal:
+    // sub-partition q reads row 32 q + l's scales from column 4 j + q of A's
+    // chunk j, so warp q stores word q there and nothing else (checked by the
+    // GEMM parity tests: with any of these words missing the results differ).
     if constexpr (C::SCALED) {
       const uint32_t q = static_cast<uint32_t>(warp & 3);
       const uint32_t leader_full0 = map_to_cta(full_bar(0), 0);
-      constexpr int NCH = C::SF_CHUNKS * (1 + C::NRB);  // A chunks, then B chunks
+      constexpr int NA = C::SF_CHUNKS;            // A chunks per stage
+      constexpr int NB = C::SF_CHUNKS * C::NRB;   // B chunks per stage
       int r = 0, n = 0;
       uint32_t rph = 0, nph = 0;
       for (int g = 0; g < total_kb; ++g) {
         if (!mbar_wait_bounded(sf_full_bar(r), rph)) break;
         const uint32_t slot = sf_base + r * C::SF_SLOT_BYTES;
-        uint32_t v[NCH * 4];
+        uint32_t va[NA], vb[NB * 4];
 #pragma unroll
-        for (int i = 0; i < NCH; ++i) {
-          // TMEM order: A j, then B (j, c) MMA-major; the slot holds B as (c, j)
-          int off;
-          if (i < C::SF_CHUNKS) {
-            off = i * 512;
-          } else {
-            const int jb = (i - C::SF_CHUNKS) / C::NRB, cb = (i - C::SF_CHUNKS) % C::NRB;
-            off = C::SFA_BYTES + (cb * C::SF_CHUNKS + jb) * 512;
-          }
+        for (int i = 0; i < NA; ++i)
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(va[i]) : "r"(slot + i * 512 + lane * 16 + q * 4));
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          // TMEM order is MMA-major (j, c); the slot holds B as (c, j)
+          const int jb = i / C::NRB, cb = i % C::NRB;
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(v[4 * i]), "=r"(v[4 * i + 1]), "=r"(v[4 * i + 2]), "=r"(v[4 * i + 3])
-                       : "r"(slot + off + lane * 16));
+                       : "=r"(vb[4 * i]), "=r"(vb[4 * i + 1]), "=r"(vb[4 * i + 2]), "=r"(vb[4 * i + 3])
+                       : "r"(slot + C::SFA_BYTES + (cb * C::SF_CHUNKS + jb) * 512 + lane * 16));
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(sf_empty_bar(r));  // slot read: the loader may refill it
@@ -387,18 +388,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         if (g >= S && !mbar_wait_bounded(empty_bar(n), nph ^ 1u)) break;
         tc_fence_after();
         const uint32_t t = tmem_base + (q * 32u << 16) + C::SF_COL + n * C::SF_SET_COLS;
-        if constexpr (NCH * 4 % 16 == 0) {
 #pragma unroll
-          for (int i = 0; i < NCH * 4 / 16; ++i) {
+        for (int i = 0; i < NA; ++i) tmem_st_32x32b_x1(t + 4 * i + q, va[i]);
+        if constexpr (NB * 4 % 16 == 0) {
+#pragma unroll
+          for (int i = 0; i < NB * 4 / 16; ++i) {
             uint32_t w[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) w[k] = v[16 * i + k];
-            tmem_st_32x32b_x16(t + 16 * i, w);
+            for (int k = 0; k < 16; ++k) w[k] = vb[16 * i + k];
+            tmem_st_32x32b_x16(t + C::SFB_OFF + 16 * i, w);
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < NCH; ++i)
-            tmem_st_32x32b_x4(t + 4 * i, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < NB; ++i)
+            tmem_st_32x32b_x4(t + C::SFB_OFF + 4 * i, vb[4 * i], vb[4 * i + 1], vb[4 * i + 2], vb[4 * i + 3]);
         }
         tc_wait_st();
         tc_fence_before();

@@ -406,6 +406,10 @@ __device__ __forceinline__ void reg_fence32(uint32_t* r) {
 }
 
 // Store 4 consecutive 32-bit columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_st_32x32b_x1(uint32_t taddr, uint32_t a) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(a) : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c,
                                                   uint32_t d) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a),
