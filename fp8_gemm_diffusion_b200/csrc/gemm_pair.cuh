@@ -14,7 +14,8 @@
 //               into this CTA's ring; completions land on the even CTA's full
 //               barrier (cta_group::2 loads, no multicast).
 //   warps 1, 3  on the even CTA lane 0 of each issues every other stage's
-//               MMAs (one thread cannot issue them fast enough) and commits
+//               MMAs (one thread cannot issue them fast enough; all of them
+//               accumulate, so their order does not matter) and commits
 //               to both CTAs' barriers (multicast commit): stage free (its A/B
 //               slot and its scale set) and accumulator full.  A stage's
 //               commit is issued after that thread's next wait, so the wait
@@ -29,9 +30,11 @@
 //               they arrive on the even CTA's full barrier of the stage, which
 //               thus completes when A, B and all scales are in place.
 //   warps 8-15  epilogue, sub-partition warp % 4, column half (warp / 4) % 2:
-//               the warp's accumulator columns into registers, release of the
-//               accumulator, then alpha, bias, bf16, 64-byte swizzled staging
-//               and TMA stores of 32 x 32 sub-tiles.
+//               the warp's accumulator columns into registers, zeros written
+//               in their place (every MMA accumulates), release of the
+//               accumulator, then alpha * acc + bias (fp32 bias row in shared
+//               memory), bf16, 64-byte swizzled staging and TMA stores of
+//               32 x 32 sub-tiles.
 // Tiles are visited along the smaller operand first (pair_tile_coords).
 // Every wait is bounded (ptx.cuh); a timed-out role stops, loads and MMAs in
 // flight are drained, and both CTAs free tensor memory together.
@@ -88,7 +91,7 @@ struct PairCfg {
   static constexpr int EPI_BYTES = EPI_WARPS * 32 * EPI_SUB * 2;
   static constexpr int EPI_BIAS_BYTES = EPI_WARPS * EPI_COLS * 4;  // each warp's bias columns, fp32
   // registers: launched with 65536 / 512 = 128 per thread, then rebalanced
-  static constexpr int REGS_CTRL = 56, REGS_SFW = 80, REGS_EPI = 184;
+  static constexpr int REGS_CTRL = 72, REGS_SFW = 72, REGS_EPI = 184;
   static constexpr int BAR_BYTES = 512;
   static constexpr int STAGES_FIT =
       (232448 - 1024 - BAR_BYTES - EPI_BYTES - EPI_BIAS_BYTES - SF_SLOTS * SF_SLOT_BYTES) /
@@ -256,14 +259,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
     }
   } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------------ MMA issuers
-    // Lane 0 of warps 1 and 3 (two schedulers) share a tile's stages: one
-    // thread cannot issue the M=256 block-scaled MMAs fast enough to keep the
-    // tensor pipe busy (each tcgen05.mma takes ~100 cycles to issue, a stage's
-    // four execute in 512 at the full FP4 rate), two can.  Warp 1 issues
-    // stages 0 and 1 and then the odd ones, warp 3 the even ones from 2 on.
-    // Only stage 0 overwrites the accumulator; every other MMA accumulates, so
-    // warp 3 waits for stage 0 to complete before its first stage (meanwhile
-    // the pipe runs stage 1).  Each issuer commits its own stages; the
+    // Lane 0 of warps 1 and 3 (two schedulers) issue alternate stages of each
+    // tile: one thread cannot issue the M=256 block-scaled MMAs fast enough to
+    // keep the tensor pipe busy (each tcgen05.mma takes ~100 cycles to issue,
+    // a stage's four execute in 512 at the full FP4 rate), two can.  Every MMA
+    // accumulates: the epilogue zeroes the accumulator when it has read it
+    // (and once before the first tile), so the two threads' MMAs need no
+    // order among themselves.  Each issuer commits its own stages; the
     // accumulator-full and drain barriers count one commit from each.
     const int me = warp == 1 ? 0 : 1;
     if (lane == 0 && rank == 0) {
@@ -278,22 +280,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         int mt, nt;
         pair_tile_coords(tile, m_tiles, n_tiles, n_fast, mt, nt);
         const uint32_t sfb_shift = ((nt * BN) & 127) >> 5;
-        // the accumulator is single-buffered: wait until the epilogue has read the
-        // last tile (both issuers, so neither commits for this tile too early)
-        if (!mbar_wait_bounded(tempty_bar, acc_ph ^ 1u)) { ok = false; break; }
+        // the accumulator is single-buffered: wait until the epilogue has read and
+        // zeroed it (both issuers, so neither commits for this tile too early)
+        if (!mbar_wait_bounded(tempty_bar, acc_ph)) { ok = false; break; }
         acc_ph ^= 1u;
         tc_fence_after();
-        const int s_first = s;  // the tile's first stage: its slot and phase
-        const uint32_t ph_first = ph;
         for (int kb = 0; kb < num_kb; ++kb) {
           const int cs = s;
           const uint32_t cph = ph;
           if (++s == S) { s = 0; ph ^= 1u; }
-          const int owner = (kb < 2 || (kb & 1)) ? 0 : 1;
-          if (owner != me) continue;  // the other issuer's stage
-          // warp 3's first stage of the tile: wait until the accumulator-
-          // overwriting stage 0 has completed
-          if (kb == 2 && !mbar_wait_bounded(empty_bar(s_first), ph_first)) { ok = false; break; }
+          if ((kb & 1) != me) continue;  // the other issuer's stage
           if (!mbar_wait_bounded(full_bar(cs), cph)) { ok = false; break; }
           // this thread's previous stage is committed after this wait, since a
           // barrier wait issued right behind a commit takes a few hundred cycles longer
@@ -308,7 +304,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
 #pragma unroll
           for (int j = 0; j < C::MMAS; ++j) {
             if (j < nmma) {
-              const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
+              const uint32_t accum = 1u;  // the accumulator starts zeroed
               const uint64_t koff = static_cast<uint64_t>(2 * j);  // 32 bytes of K per MMA
               if constexpr (F == Fmt::NVFP4) {
                 mma_pair_nvfp4(tmem_base, adesc + koff, bdesc + koff, idesc, sf + 4 * j,
@@ -445,6 +441,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
     const bool has_bias = args.bias != nullptr;
     const bool bias_vec = has_bias && (reinterpret_cast<uintptr_t>(args.bias) & 15u) == 0;
     const uint32_t bias_buf = bias_base + (warp - C::EPI_WARP0) * (C::EPI_COLS * 4);
+    // the MMAs only accumulate: this warp's accumulator columns start at zero
+    // (and are zeroed again after every read); the arrival is the accumulator's
+    // first "free" signal
+#pragma unroll
+    for (int g = 0; g < C::EPI_COLS / 32; ++g)
+      tmem_st_32x32b_x32_zero(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + h * C::EPI_COLS + g * 32);
+    tc_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_remote(leader_tempty);
     for (int i_tile = 0; i_tile < my_tiles; ++i_tile) {
       const int tile = pair + i_tile * num_pairs;
       int mt, nt;
@@ -481,7 +487,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       __syncwarp();
       if (!mbar_wait_bounded(tfull_bar, i_tile & 1)) break;
       tc_fence_after();
-      // all of this warp's accumulator columns into registers, then release the accumulator
+      // all of this warp's accumulator columns into registers, zeros in their
+      // place, then release the accumulator
       uint32_t r[C::EPI_COLS];
       const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + h * C::EPI_COLS;
 #pragma unroll
@@ -489,6 +496,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       tc_wait_ld();
 #pragma unroll
       for (int g = 0; g < C::EPI_COLS / 32; ++g) reg_fence32(r + 32 * g);
+#pragma unroll
+      for (int g = 0; g < C::EPI_COLS / 32; ++g) tmem_st_32x32b_x32_zero(t_cols + g * 32);
+      tc_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(leader_tempty);  // accumulator may be overwritten
