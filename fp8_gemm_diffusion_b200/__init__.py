@@ -64,7 +64,8 @@ class mxq_weight(ctypes.Structure):
 
 
 class mxq_linear_opts(ctypes.Structure):
-    _fields_ = [("min_dim", _i64)]
+    _fields_ = [("min_dim", _i64), ("gemm_event_start", ctypes.c_void_p),
+                ("gemm_event_end", ctypes.c_void_p)]
 
 
 def _proto(name, restype, *argtypes):
@@ -221,8 +222,15 @@ def weight_prepare(fmt, w, N, K, bias, keep_bf16, storage, storage_bytes, stream
     return out
 
 
-def _opts(min_dim):
-    return None if min_dim is None else ctypes.byref(mxq_linear_opts(int(min_dim)))
+def _opts(min_dim, gemm_events=None):
+    """mxq_linear_opts; gemm_events: (start, end) torch.cuda.Event pair recorded
+    around the GEMM launch, or None."""
+    if min_dim is None and gemm_events is None:
+        return None
+    o = mxq_linear_opts(int(min_dim or 0))
+    if gemm_events is not None:
+        o.gemm_event_start, o.gemm_event_end = (ev.cuda_event for ev in gemm_events)
+    return ctypes.byref(o)
 
 
 def linear_path(w: mxq_weight, M: int, min_dim=None) -> int:
@@ -238,9 +246,9 @@ def linear_workspace_bytes(M: int, K: int, fmt) -> int:
     return _linear_workspace_bytes(M, K, _fmt(fmt))
 
 
-def linear(w: mxq_weight, x, M, y, ws, ws_bytes, min_dim=None, stream=None) -> None:
-    _check(_linear(ctypes.byref(w), _addr(x), M, _addr(y), _addr(ws), ws_bytes, _opts(min_dim),
-                   _stream(stream)), "mxq_linear")
+def linear(w: mxq_weight, x, M, y, ws, ws_bytes, min_dim=None, stream=None, gemm_events=None) -> None:
+    _check(_linear(ctypes.byref(w), _addr(x), M, _addr(y), _addr(ws), ws_bytes,
+                   _opts(min_dim, gemm_events), _stream(stream)), "mxq_linear")
 
 
 def linear_noalloc(w: mxq_weight, x, M, y, min_dim=None, stream=None) -> None:

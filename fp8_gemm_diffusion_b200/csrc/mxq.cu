@@ -638,10 +638,22 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
   if (N % 8 != 0) return MXQ_ERR_ALIGNMENT;  // y rows are N elements apart
   const int path = mxq_linear_path(w, M, opts);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  if (opts != nullptr) {
+    if ((opts->gemm_event_start == nullptr) != (opts->gemm_event_end == nullptr))
+      return MXQ_ERR_INVALID_ARG;
+    ev0 = static_cast<cudaEvent_t>(opts->gemm_event_start);
+    ev1 = static_cast<cudaEvent_t>(opts->gemm_event_end);
+  }
   if (path == MXQ_BF16) {
     if (M > 0 && N > 0 && w->w_bf16 == nullptr) return MXQ_ERR_INVALID_ARG;
-    return mxq_gemm_blockscaled(MXQ_BF16, M, N, K, x_bf16, nullptr, nullptr, w->w_bf16, nullptr,
-                                nullptr, w->bias_bf16, y_bf16, N, stream);
+    cudaError_t e;
+    if (ev0 != nullptr && (e = cudaEventRecord(ev0, s)) != cudaSuccess) return cuda_fail(e);
+    st = mxq_gemm_blockscaled(MXQ_BF16, M, N, K, x_bf16, nullptr, nullptr, w->w_bf16, nullptr,
+                              nullptr, w->bias_bf16, y_bf16, N, stream);
+    if (st == MXQ_OK && ev1 != nullptr && (e = cudaEventRecord(ev1, s)) != cudaSuccess)
+      return cuda_fail(e);
+    return st;
   }
   const mxq_format f = static_cast<mxq_format>(path);
   if (w->codes == nullptr || w->sf == nullptr) return MXQ_ERR_INVALID_ARG;
@@ -679,8 +691,13 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
     if ((st = launch_quant_mxfp8(x_bf16, M, K, K, codes, sf, s, sms)) != MXQ_OK) return st;
   }
   if ((st = get_encoder()) != MXQ_OK) return st;
-  return launch_gemm(f, dev, sms, M, N, K, codes, sf, g, w->codes, w->sf, w->g_dev, w->bias_bf16,
-                     y_bf16, N, s);
+  cudaError_t e;
+  if (ev0 != nullptr && (e = cudaEventRecord(ev0, s)) != cudaSuccess) return cuda_fail(e);
+  st = launch_gemm(f, dev, sms, M, N, K, codes, sf, g, w->codes, w->sf, w->g_dev, w->bias_bf16,
+                   y_bf16, N, s);
+  if (st == MXQ_OK && ev1 != nullptr && (e = cudaEventRecord(ev1, s)) != cudaSuccess)
+    return cuda_fail(e);
+  return st;
 }
 
 int mxq_linear_kernel_count(const mxq_weight* w, int64_t M, const mxq_linear_opts* opts) {

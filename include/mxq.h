@@ -191,7 +191,12 @@ mxq_status mxq_weight_prepare(mxq_format f, const void* w_bf16, int64_t N, int64
 
 /* Options of mxq_linear.  A NULL pointer means the defaults. */
 typedef struct mxq_linear_opts {
-  int64_t min_dim;   /* bf16 when min(M,K,N) < min_dim; 0 -> 1024 (the article's rule) */
+  int64_t min_dim;          /* bf16 when min(M,K,N) < min_dim; 0 -> 1024 (the article's rule) */
+  void* gemm_event_start;   /* optional cudaEvent_t (NULL: none): mxq_linear records it on the
+                               stream right before its GEMM launch and gemm_event_end right
+                               after, so a caller can time the GEMM inside a step.  Both or
+                               neither; the events stay the caller's. */
+  void* gemm_event_end;
 } mxq_linear_opts;
 
 /*

@@ -144,3 +144,18 @@ def test_linear_kernel_count_host_cases():
         # the NVFP4 choice (one or two quantiser kernels) depends on the SM count
         w = mxq.mxq_weight(format=mxq.NVFP4, keep_bf16=0, N=1024, K=1024)
         assert mxq.linear_kernel_count(w, 4096) == -1
+
+
+class _FakeEvent:
+    """Stands in for a torch.cuda.Event: only its handle is passed (never used)."""
+
+    def __init__(self, handle):
+        self.cuda_event = handle
+
+
+def test_linear_rejects_half_an_event_pair():
+    w = mxq.mxq_weight(format=mxq.NVFP4, keep_bf16=0, N=4096, K=4096, w_bf16=A16, bias_bf16=None,
+                       codes=A16, sf=A16, g_dev=A16, amax_dev=A16)
+    need = mxq.linear_workspace_bytes(4096, 4096, "nvfp4")
+    half = (_FakeEvent(0x1000), _FakeEvent(0))
+    assert _st(mxq.linear, w, A16, 4096, A16, A16, need, None, None, half) == mxq.ERR_INVALID_ARG

@@ -132,3 +132,24 @@ def test_kernel_count_matches_the_path_taken():
     assert mxq.linear_kernel_count(w.handle, 4608, min_dim=1) == 2   # single pass + GEMM
     w = _weight(4096)
     assert mxq.linear_kernel_count(w.handle, 4608, min_dim=1) == 3   # amax + quantise + GEMM
+
+
+def test_gemm_events_bracket_the_gemm():
+    # the optional event pair of mxq_linear_opts brackets the GEMM launch: its
+    # interval is positive and inside the interval of the whole call
+    w = _weight(3072, N=1024)
+    A = workloads.random_case(4608, 3072, 8, "nvfp4", seed=3).A.to(DEV)
+    nbytes = mxq.linear_workspace_bytes(4608, 3072, "nvfp4")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
+    y = torch.empty(4608, 1024, dtype=torch.bfloat16, device=DEV)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in ev:
+        e.record()
+    torch.cuda.synchronize()
+    ev[0].record()
+    mxq.linear(w.handle, A, 4608, y, ws, nbytes, min_dim=1, gemm_events=(ev[1], ev[2]))
+    ev[3].record()
+    torch.cuda.synchronize()
+    gemm = ev[1].elapsed_time(ev[2])
+    assert 0.0 < gemm <= ev[0].elapsed_time(ev[3])
+    assert mxq.get_device_error() == mxq.OK
