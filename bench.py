@@ -1,7 +1,7 @@
 """Benchmark of the microscaled linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3|c2|c4|c1]
-                    [--impl mxq|reference]
+                    [--impl mxq|reference] [--shape M,K,N --fmt nvfp4|mxfp8]
 
 A step is one pass of the whole hot path over one batch of synthetic input:
 for NVFP4, activation amax -> NVFP4 quantisation -> block-scaled GEMM with the
@@ -157,7 +157,11 @@ def run_gpu(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    case = workloads.make_case(args.workload)
+    if args.shape:
+        Ms, Ks, Ns = (int(v) for v in args.shape.split(","))
+        case = workloads.random_case(Ms, Ks, Ns, args.fmt, seed=0)
+    else:
+        case = workloads.make_case(args.workload)
     fmt = case.fmt
     M, K, N = case.M, case.K, case.N
     flops = 2.0 * M * N * K
@@ -286,6 +290,10 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     quant_pub_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
 
+    # bf16 tensor-core baseline in the same run: cuBLAS (torch.addmm) on the
+    # same shape, bias and rotating buffers, timed the same way
+    bf16_ms = bf16_baseline_ms(sets, W, bias, M, N, stream, args.warmup, min(args.steps, 500), dev, dist)
+
     # end to end through the public call with host buffers
     e2e = run_e2e(mxq, case, base_w, dev, stream, args, dist)
 
@@ -295,6 +303,7 @@ def run_gpu(args, rank, world, local_rank):
     peak_burst = peaks["bf16"] * NOMINAL_RATIO[fmt]
     achieved = flops / (gemm_ms * 1e-3) / 1e12
     value = whole_job_tflops(world, args.steps, flops, total_ms)
+    bf16_tflops = whole_job_tflops(world, 1, flops, bf16_ms)
     step_ms = total_ms / args.steps
     qbytes = M * K * 2 + mxq.codes_bytes(M, K, fmt) + mxq.sf_bytes(M, K, fmt)
     nominal = {"nvfp4": 9000.0, "mxfp8": 4500.0}[fmt]
@@ -342,11 +351,41 @@ def run_gpu(args, rank, world, local_rank):
             "traffic": GEMM_TRAFFIC_BYTES.get(case.name),
             "traffic_unit": "bytes per launch (ncu dram read + write)",
         },
+        "bf16_baseline": {
+            "impl": "torch.addmm bf16 (cuBLAS), same shape, bias and buffers",
+            "value": round(bf16_tflops, 2), "unit": UNIT,
+            "ms_per_step": round(bf16_ms, 5),
+            "speedup_of_value": round(value / bf16_tflops, 3),
+        },
         "clocks": sampler.summary(),
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
     }
     return result
+
+
+def bf16_baseline_ms(sets, W, bias, M, N, stream, warmup, steps, dev, dist):
+    """Average step time of y = x W^T + bias in bf16 through cuBLAS (torch.addmm),
+    over the bench's rotating activation / output buffers."""
+    Wt = W.t()
+    b = bias if bias is not None else torch.zeros(N, dtype=torch.bfloat16, device=W.device)
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            st = sets[i % len(sets)]
+            torch.addmm(b, st["x"], Wt, out=st["y"])
+        torch.cuda.synchronize()
+        if dist:
+            import torch.distributed as tdist
+            tdist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            st = sets[i % len(sets)]
+            torch.addmm(b, st["x"], Wt, out=st["y"])
+        e1.record(stream)
+        torch.cuda.synchronize()
+    return max_over_ranks(e0.elapsed_time(e1), dev) / steps
 
 
 def run_e2e(mxq, case, base_w, dev, stream, args, dist):
@@ -444,6 +483,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4"])
     ap.add_argument("--impl", default="mxq", choices=["mxq", "reference"])
+    ap.add_argument("--shape", default=None,
+                    help="M,K,N of a seeded random layer instead of a named workload (profiling)")
+    ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp8"], help="format for --shape")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -485,7 +527,7 @@ def main():
                                  device_id=torch.device("cuda", local_rank))
     try:
         result = run_gpu(args, rank, world, local_rank)
-        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.shape:
             result["cpu_baseline"] = run_oracle_sample(args.workload)
         if rank == 0:
             print(json.dumps(result))

@@ -13,14 +13,11 @@
 //   warp 0      A/B producer: each stage's 128 rows of A and BN/2 rows of B
 //               into this CTA's ring; completions land on the even CTA's full
 //               barrier (cta_group::2 loads, no multicast).
-//   warps 1, 3  on the even CTA lane 0 of each issues every other stage's
-//               MMAs (one thread cannot issue them fast enough; all of them
-//               accumulate, so their order does not matter) and commits
-//               to both CTAs' barriers (multicast commit): stage free (its A/B
-//               slot and its scale set) and accumulator full.  A stage's
-//               commit is issued after that thread's next wait, so the wait
-//               never follows a commit.  Warp 1 also owns the tensor memory
-//               (cta_group::2 allocation).
+//   warp 1      tensor memory (cta_group::2 allocation); on the even CTA one
+//               lane issues the MMAs and commits to both CTAs' barriers
+//               (multicast commit): stage free (its A/B slot and its scale
+//               set) and accumulator full.  A stage's commit is issued after
+//               the next stage's wait, so the wait never follows a commit.
 //   warp 2      scale loader: the scale chunks of each stage (A's 128 rows and
 //               all BN columns of B: each CTA's tensor memory needs B's) into
 //               a separate ring that runs ahead of the A/B ring.
@@ -30,11 +27,9 @@
 //               they arrive on the even CTA's full barrier of the stage, which
 //               thus completes when A, B and all scales are in place.
 //   warps 8-15  epilogue, sub-partition warp % 4, column half (warp / 4) % 2:
-//               the warp's accumulator columns into registers, zeros written
-//               in their place (every MMA accumulates), release of the
-//               accumulator, then alpha * acc + bias (fp32 bias row in shared
-//               memory), bf16, 64-byte swizzled staging and TMA stores of
-//               32 x 32 sub-tiles.
+//               the warp's accumulator columns into registers, release of the
+//               accumulator, then alpha, bias, bf16, 64-byte swizzled staging
+//               and TMA stores of 32 x 32 sub-tiles.
 // Tiles are visited along the smaller operand first (pair_tile_coords).
 // Every wait is bounded (ptx.cuh); a timed-out role stops, loads and MMAs in
 // flight are drained, and both CTAs free tensor memory together.
@@ -72,7 +67,7 @@ struct PairCfg {
   static constexpr int SFB_BYTES = NRB * SF_CHUNKS * 512;
   static constexpr uint32_t SF_TX = SFA_BYTES + SFB_BYTES;  // this CTA's scales
   static constexpr int SF_SLOT_BYTES = SCALED ? (SFA_BYTES + SFB_BYTES + 1023) / 1024 * 1024 : 0;
-  static constexpr int SF_SLOTS = SCALED ? (F == Fmt::NVFP4 ? 4 : 6) : 0;
+  static constexpr int SF_SLOTS = SCALED ? (F == Fmt::NVFP4 ? 4 : 8) : 0;
   // tensor memory: the accumulator (BN columns), then one scale set per A/B
   // stage (A chunks, then B chunks in MMA-major order, 4 columns each)
   static constexpr int SF_SET_COLS = (SF_CHUNKS + NRB * SF_CHUNKS) * 4;
@@ -80,7 +75,7 @@ struct PairCfg {
   static constexpr int SFB_OFF = SF_CHUNKS * 4;
   static constexpr int TMEM_COLS = 512;
   static constexpr int NS_FIT = SCALED ? (TMEM_COLS - BN) / SF_SET_COLS : 64;
-  // warp roles, one warpgroup each for (producer, MMA issuer, scale loader, MMA issuer),
+  // warp roles, one warpgroup each for (producer, MMA, scale loader, spare),
   // the scale writers and the two halves of the epilogue
   static constexpr int SF_WARP0 = 4;   // warps 4-7, one per tensor-memory sub-partition
   static constexpr int SF_WARPS = 4;
@@ -89,13 +84,14 @@ struct PairCfg {
   static constexpr int EPI_COLS = BN / 2;   // accumulator columns per epilogue warp
   static constexpr int EPI_SUB = 32;        // staging sub-tile: 32 rows x 32 columns (64-byte rows)
   static constexpr int EPI_BYTES = EPI_WARPS * 32 * EPI_SUB * 2;
-  static constexpr int EPI_BIAS_BYTES = EPI_WARPS * EPI_COLS * 4;  // each warp's bias columns, fp32
-  // registers: launched with 65536 / 512 = 128 per thread, then rebalanced
-  static constexpr int REGS_CTRL = 72, REGS_SFW = 72, REGS_EPI = 184;
+  // registers: launched with 65536 / 512 = 128 per thread, then rebalanced.
+  // Keep the margins: with 72 for the scale writers (ptxas reported no
+  // spills) repeated launches produced wrong scales in whole 32-row slices,
+  // i.e. a writer warp lost register contents to the epilogue's increase.
+  static constexpr int REGS_CTRL = 56, REGS_SFW = 80, REGS_EPI = 184;
   static constexpr int BAR_BYTES = 512;
   static constexpr int STAGES_FIT =
-      (232448 - 1024 - BAR_BYTES - EPI_BYTES - EPI_BIAS_BYTES - SF_SLOTS * SF_SLOT_BYTES) /
-      STAGE_BYTES;
+      (232448 - 1024 - BAR_BYTES - EPI_BYTES - SF_SLOTS * SF_SLOT_BYTES) / STAGE_BYTES;
   static constexpr int STAGES_MIN = STAGES_FIT < NS_FIT ? STAGES_FIT : NS_FIT;
   static constexpr int STAGES = STAGES_MIN > 8 ? 8 : STAGES_MIN;
   // arrivals that complete a stage's full barrier besides the A/B bytes: the
@@ -103,7 +99,7 @@ struct PairCfg {
   static constexpr int FULL_ARRIVALS = 1 + (SCALED ? 2 * SF_WARPS : 0);
   static_assert(STAGES >= 2, "shared / tensor memory");
   static constexpr int SMEM_BYTES =
-      1024 + STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + EPI_BYTES + EPI_BIAS_BYTES + BAR_BYTES;
+      1024 + STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + EPI_BYTES + BAR_BYTES;
   static constexpr int THREADS = 512;
   static_assert(128 * (REGS_CTRL + REGS_SFW) + 256 * REGS_EPI <= 65536, "register split");
 };
@@ -158,8 +154,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
   uint8_t* const base_ptr = smem_raw + (base - raw_addr);
   const uint32_t sf_base = base + S * C::STAGE_BYTES;
   const uint32_t epi_base = sf_base + R * C::SF_SLOT_BYTES;
-  const uint32_t bias_base = epi_base + C::EPI_BYTES;
-  const uint32_t bar_base = bias_base + C::EPI_BIAS_BYTES;
+  const uint32_t bar_base = epi_base + C::EPI_BYTES;
   // barriers: [full S][empty S][sf_full R][sf_empty R][tfull][tempty][drain]
   auto full_bar = [&](int s) { return bar_base + 8u * s; };  // even CTA: A/B landed, scales written
   auto empty_bar = [&](int s) { return bar_base + 8u * (S + s); };          // both: A/B stage free
@@ -195,9 +190,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       mbar_init(sf_full_bar(r), 1);
       mbar_init(sf_empty_bar(r), C::SF_WARPS);
     }
-    mbar_init(tfull_bar, 2);  // one commit from each MMA issuer
+    mbar_init(tfull_bar, 1);
     mbar_init(tempty_bar, 2 * C::EPI_WARPS);
-    mbar_init(drain_bar, 2);
+    mbar_init(drain_bar, 1);
     fence_barrier_init();
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
@@ -257,19 +252,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         }
       }
     }
-  } else if (warp == 1 || warp == 3) {
-    // ------------------------------------------------------------ MMA issuers
-    // Lane 0 of warps 1 and 3 (two schedulers) issue alternate stages of each
-    // tile: one thread cannot issue the M=256 block-scaled MMAs fast enough to
-    // keep the tensor pipe busy (each tcgen05.mma takes ~100 cycles to issue,
-    // a stage's four execute in 512 at the full FP4 rate), two can.  Every MMA
-    // accumulates: the epilogue zeroes the accumulator when it has read it
-    // (and once before the first tile), so the two threads' MMAs need no
-    // order among themselves.  Each issuer commits its own stages; the
-    // accumulator-full and drain barriers count one commit from each.
-    const int me = warp == 1 ? 0 : 1;
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // (one thread: keep the per-stage work to a few instructions)
     if (lane == 0 && rank == 0) {
-      int s = 0, pend = -1;  // pend: this thread's stage whose MMAs are issued but not committed
+      int s = 0, pend = -1;  // pend: stage whose MMAs are issued but not committed
       uint32_t ph = 0, acc_ph = 0;
       bool ok = true;
       const uint64_t adesc0 = desc_kmajor_sw128(base);
@@ -280,23 +267,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         int mt, nt;
         pair_tile_coords(tile, m_tiles, n_tiles, n_fast, mt, nt);
         const uint32_t sfb_shift = ((nt * BN) & 127) >> 5;
-        // the accumulator is single-buffered: wait until the epilogue has read and
-        // zeroed it (both issuers, so neither commits for this tile too early)
-        if (!mbar_wait_bounded(tempty_bar, acc_ph)) { ok = false; break; }
+        // the accumulator is single-buffered: wait until the epilogue has read the last tile
+        if (!mbar_wait_bounded(tempty_bar, acc_ph ^ 1u)) { ok = false; break; }
         acc_ph ^= 1u;
         tc_fence_after();
         for (int kb = 0; kb < num_kb; ++kb) {
-          const int cs = s;
-          const uint32_t cph = ph;
-          if (++s == S) { s = 0; ph ^= 1u; }
-          if ((kb & 1) != me) continue;  // the other issuer's stage
-          if (!mbar_wait_bounded(full_bar(cs), cph)) { ok = false; break; }
-          // this thread's previous stage is committed after this wait, since a
-          // barrier wait issued right behind a commit takes a few hundred cycles longer
+          if (!mbar_wait_bounded(full_bar(s), ph)) { ok = false; break; }
+          // the previous stage's commit: after this wait, since a barrier wait
+          // issued right behind a commit takes a few hundred cycles longer
           if (pend >= 0) tc_commit_pair(empty_bar(pend));
           tc_fence_after();
-          const uint64_t adesc = adesc0 + DSTEP * cs, bdesc = bdesc0 + DSTEP * cs;
-          const uint32_t sf = tmem_base + C::SF_COL + cs * C::SF_SET_COLS;
+          const uint64_t adesc = adesc0 + DSTEP * s, bdesc = bdesc0 + DSTEP * s;
+          const uint32_t sf = tmem_base + C::SF_COL + s * C::SF_SET_COLS;
           int nmma = C::MMAS;
           if constexpr (F == Fmt::NVFP4) {
             if (kb == num_kb - 1) nmma = K / 64 - kb * C::MMAS;  // K % 256 != 0: partial last stage
@@ -304,7 +286,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
 #pragma unroll
           for (int j = 0; j < C::MMAS; ++j) {
             if (j < nmma) {
-              const uint32_t accum = 1u;  // the accumulator starts zeroed
+              const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
               const uint64_t koff = static_cast<uint64_t>(2 * j);  // 32 bytes of K per MMA
               if constexpr (F == Fmt::NVFP4) {
                 mma_pair_nvfp4(tmem_base, adesc + koff, bdesc + koff, idesc, sf + 4 * j,
@@ -319,7 +301,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
               }
             }
           }
-          pend = cs;  // committed (A/B slot and scale set free) after this thread's next wait
+          pend = s;  // committed (A/B slot and scale set s free) after the next wait
+          if (++s == S) { s = 0; ph ^= 1u; }
         }
         if (pend >= 0) tc_commit_pair(empty_bar(pend));
         pend = -1;
@@ -365,6 +348,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         }
       }
     }
+  } else if (warp == 3) {
+    // spare warp of the control warpgroup
   }
   } else if (warp < C::EPI_WARP0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_SFW));
@@ -438,57 +423,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
     const uint32_t leader_tempty = map_to_cta(tempty_bar, 0);
     float alpha = 1.0f;
     if constexpr (F == Fmt::NVFP4) alpha = (*args.a_g) * (*args.b_g);
-    const bool has_bias = args.bias != nullptr;
-    const bool bias_vec = has_bias && (reinterpret_cast<uintptr_t>(args.bias) & 15u) == 0;
-    const uint32_t bias_buf = bias_base + (warp - C::EPI_WARP0) * (C::EPI_COLS * 4);
-    // the MMAs only accumulate: this warp's accumulator columns start at zero
-    // (and are zeroed again after every read); the arrival is the accumulator's
-    // first "free" signal
-#pragma unroll
-    for (int g = 0; g < C::EPI_COLS / 32; ++g)
-      tmem_st_32x32b_x32_zero(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + h * C::EPI_COLS + g * 32);
-    tc_wait_st();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive_remote(leader_tempty);
+    const bool bias_vec = args.bias != nullptr && (reinterpret_cast<uintptr_t>(args.bias) & 15u) == 0;
     for (int i_tile = 0; i_tile < my_tiles; ++i_tile) {
       const int tile = pair + i_tile * num_pairs;
       int mt, nt;
       pair_tile_coords(tile, m_tiles, n_tiles, n_fast, mt, nt);
       const int row0 = mt * C::BM + static_cast<int>(rank) * C::BM_CTA + q * 32;
-      const int col_w = nt * BN + h * C::EPI_COLS;  // first column of this warp
-      // this warp's bias columns as fp32 in shared memory, staged before the
-      // accumulator is ready (lane l: columns [8l, 8l + 8)); every lane later
-      // reads the same address (a broadcast), so the conversion loop needs
-      // neither shuffles nor bf16 unpacking
-      if (has_bias && lane * 8 < C::EPI_COLS) {
-        const int c0 = col_w + lane * 8;
-        uint32_t bw[4];
+      // the tile's bias, prefetched before the accumulator is ready: lane l holds
+      // columns [8l, 8l + 8) of the tile as four packed bf16 pairs
+      uint32_t bias_l[4] = {0u, 0u, 0u, 0u};
+      if (args.bias != nullptr && lane * 8 < BN) {
+        const int c0 = nt * BN + lane * 8;
         if (bias_vec && c0 + 8 <= N) {
           const uint4 u = __ldg(reinterpret_cast<const uint4*>(args.bias + c0));
-          bw[0] = u.x; bw[1] = u.y; bw[2] = u.z; bw[3] = u.w;
+          bias_l[0] = u.x; bias_l[1] = u.y; bias_l[2] = u.z; bias_l[3] = u.w;
         } else {
           const uint16_t* bs = reinterpret_cast<const uint16_t*>(args.bias);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const uint32_t lo = (c0 + 2 * e < N) ? bs[c0 + 2 * e] : 0u;
             const uint32_t hi = (c0 + 2 * e + 1 < N) ? bs[c0 + 2 * e + 1] : 0u;
-            bw[e] = lo | (hi << 16);
+            bias_l[e] = lo | (hi << 16);
           }
         }
-        const uint32_t dst = bias_buf + lane * 32;
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(bw[0] << 16),
-                     "r"(bw[0] & 0xFFFF0000u), "r"(bw[1] << 16), "r"(bw[1] & 0xFFFF0000u)
-                     : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16), "r"(bw[2] << 16),
-                     "r"(bw[2] & 0xFFFF0000u), "r"(bw[3] << 16), "r"(bw[3] & 0xFFFF0000u)
-                     : "memory");
       }
-      __syncwarp();
       if (!mbar_wait_bounded(tfull_bar, i_tile & 1)) break;
       tc_fence_after();
-      // all of this warp's accumulator columns into registers, zeros in their
-      // place, then release the accumulator
+      // all of this warp's accumulator columns into registers, then release the accumulator
       uint32_t r[C::EPI_COLS];
       const uint32_t t_cols = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + h * C::EPI_COLS;
 #pragma unroll
@@ -496,36 +457,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       tc_wait_ld();
 #pragma unroll
       for (int g = 0; g < C::EPI_COLS / 32; ++g) reg_fence32(r + 32 * g);
-#pragma unroll
-      for (int g = 0; g < C::EPI_COLS / 32; ++g) tmem_st_32x32b_x32_zero(t_cols + g * 32);
-      tc_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(leader_tempty);  // accumulator may be overwritten
+      const int col_w = nt * BN + h * C::EPI_COLS;  // first column of this warp
 #pragma unroll
       for (int sub = 0; sub < C::EPI_COLS / C::EPI_SUB; ++sub) {
         if (lane == 0) bulk_wait_group_read<0>();  // the staging sub-tile is free again
         __syncwarp();
-        // groups of 8 columns: alpha * acc + bias (one fma), bf16, one 16-byte
-        // store each into the 32 x EPI_SUB staging sub-tile (64 B rows,
-        // 64-byte swizzle: 16-byte chunk c of row l sits at chunk c ^ ((l / 2) % 4))
+        // groups of 8 columns: alpha * acc + bias, bf16, one 16-byte store each
+        // into the 32 x EPI_SUB staging sub-tile (64 B rows, 64-byte swizzle:
+        // 16-byte chunk c of row l sits at chunk c ^ ((l / 2) % 4))
 #pragma unroll
         for (int j = 0; j < C::EPI_SUB / 8; ++j) {
-          const int c8 = sub * C::EPI_SUB + j * 8;  // first column of the group in this warp's half
-          float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          if (has_bias) {
-            const uint32_t src = bias_buf + c8 * 4;
-            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                         : "=f"(b[0]), "=f"(b[1]), "=f"(b[2]), "=f"(b[3]) : "r"(src));
-            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                         : "=f"(b[4]), "=f"(b[5]), "=f"(b[6]), "=f"(b[7]) : "r"(src + 16));
-          }
+          const int grp = h * (C::EPI_COLS / 8) + sub * (C::EPI_SUB / 8) + j;  // 8-column group in the tile
+          uint32_t bw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) bw[e] = __shfl_sync(0xffffffffu, bias_l[e], grp);
           uint32_t pk[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int c = c8 + 2 * e;
-            const float v0 = fmaf(__uint_as_float(r[c]), alpha, b[2 * e]);
-            const float v1 = fmaf(__uint_as_float(r[c + 1]), alpha, b[2 * e + 1]);
+            const int c = sub * C::EPI_SUB + j * 8 + 2 * e;
+            float v0 = __uint_as_float(r[c]), v1 = __uint_as_float(r[c + 1]);
+            if constexpr (F == Fmt::NVFP4) { v0 *= alpha; v1 *= alpha; }
+            v0 += __uint_as_float(bw[e] << 16);
+            v1 += __uint_as_float(bw[e] & 0xFFFF0000u);
             const __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
             pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
           }

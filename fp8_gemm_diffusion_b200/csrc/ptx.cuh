@@ -406,15 +406,6 @@ __device__ __forceinline__ void reg_fence32(uint32_t* r) {
 }
 
 // Store 4 consecutive 32-bit columns of this warp's 32 lanes.
-// 32 lanes x 32 columns of zeros (one zero register for every element).
-__device__ __forceinline__ void tmem_st_32x32b_x32_zero(uint32_t taddr) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
-      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
-      "r"(0u)
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_st_32x32b_x1(uint32_t taddr, uint32_t a) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(a) : "memory");
 }
