@@ -20,10 +20,11 @@
 // Conversions use the hardware cvt.rn.satfinite instructions (RNE, finite
 // overflow saturates to the largest magnitude, sign kept).
 //
-// Memory layout: each thread owns one 16-byte vector (8 bf16) of a row; the
-// 2 (NVFP4) or 4 (MXFP8) lanes of a block combine their maxima with warp
-// shuffles; a warp reads 512 contiguous bytes per vector load.  Scale bytes
-// go straight to the tensor-core block-scaling layout (see sf_offset).
+// Memory layout: one warp per row.  NVFP4: one lane per 16-element block
+// (two 16-byte loads), so the block's scale arithmetic runs once per block;
+// MXFP8: one 16-byte vector per lane, the 4 lanes of a 32-element block
+// combine their maxima with warp shuffles.  Scale bytes go straight to the
+// tensor-core block-scaling layout (see sf_offset).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -121,6 +122,26 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
   return r;
 }
 
+// Same, allocating in L1: for a lane that reads both 16-byte halves of a
+// 32-byte sector with two loads, the second is served by L1.
+__device__ __forceinline__ uint4 ldg_nc_v4_l1(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// 16 bf16 (two 16-byte vectors) -> fp32, element 2i of a word in its low half.
+__device__ __forceinline__ void bf16x16_to_f32(const uint4& u0, const uint4& u1, float (&f)[16]) {
+  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
 // ------------------------------------------------------------------- amax
 // Work split: one warp per row (rows strided over all warps of the grid); a
 // lane owns every 32nd 16-byte vector of the row, four loads in flight.  No
@@ -204,20 +225,28 @@ __device__ __forceinline__ void zero_sf_padding(uint8_t* __restrict__ sf, int ro
   }
 }
 
-// One 16-byte vector (8 elements) of a row: lanes 2i and 2i+1 of the warp
-// hold the two halves of one 16-element block (every lane must call this).
-// Returns the 8 E2M1 codes packed; sfc receives the block's E4M3 scale code.
-__device__ __forceinline__ uint32_t nvfp4_vector(float (&f)[8], float g, float six_g,
-                                                 uint32_t& sfc) {
-  float bmax = absmax8(f);
-  bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));  // 16-element block
+// One 16-element block held by one lane (so the block-level steps -- the
+// division, the E4M3 scale, the reciprocal -- run once per block).  Returns
+// the 16 E2M1 codes (element 2i in the low nibble of byte i); sfc receives
+// the block's E4M3 scale code.
+__device__ __forceinline__ uint2 nvfp4_block16(float (&f)[16], float g, float six_g,
+                                               uint32_t& sfc) {
+  float bmax = fabsf(f[0]);
+#pragma unroll
+  for (int i = 1; i < 16; ++i) bmax = fmaxf(bmax, fabsf(f[i]));
   sfc = cvt_e4m3x2(bmax / six_g, 0.0f) & 0xFFu;
   const float s = e4m3_value(sfc) * g;
   const float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
+  float lo[8], hi[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) f[i] = f[i] * inv;
-  return cvt_e2m1x8(f);
+  for (int i = 0; i < 8; ++i) {
+    lo[i] = f[i] * inv;
+    hi[i] = f[8 + i] * inv;
+  }
+  return make_uint2(cvt_e2m1x8(lo), cvt_e2m1x8(hi));
 }
+
+constexpr unsigned long long kKeyMask = 0xFFFFFFFF00000000ull;
 
 // amax_in: n_amax values whose max is the tensor's amax (1 value, or the
 // per-block partials of amax_kernel).
@@ -239,30 +268,34 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (kQuantThreads / 32);
-  const int vpr = k >> 3;  // even: k is a multiple of 16
-  const int c4 = k >> 6;   // 4-column scale groups per row
+  const int bpr = k >> 4;  // 16-element blocks per row, one per lane per step
+  const uint32_t c4 = static_cast<uint32_t>(k >> 6);  // 4-column scale groups per row
   for (int r = blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
     const __nv_bfloat16* row = x + static_cast<int64_t>(r) * ld;
-    uint32_t* crow = reinterpret_cast<uint32_t*>(codes + static_cast<int64_t>(r) * (k >> 1));
-    for (int v0 = lane; v0 - lane < vpr; v0 += 32 * kQuantUnroll) {
-      uint4 u[kQuantUnroll];
+    uint2* crow = reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * (k >> 1));
+    // this row's scale bytes: 512-byte tile (r / 128, c / 4), byte (r % 32) * 16 + (r / 32 % 4) * 4 + c % 4
+    uint8_t* sf_row = sf + static_cast<int64_t>(r >> 7) * c4 * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
+    for (int c0 = lane; c0 < bpr; c0 += 32 * kQuantUnroll) {
+      uint4 u[kQuantUnroll][2];
 #pragma unroll
       for (int j = 0; j < kQuantUnroll; ++j) {
-        const int v = v0 + 32 * j;
-        u[j] = v < vpr ? ldg_nc_v4(row + v * 8) : make_uint4(0, 0, 0, 0);
+        const int c = c0 + 32 * j;
+        if (c < bpr) {
+          u[j][0] = ldg_nc_v4_l1(row + 16 * c);
+          u[j][1] = ldg_nc_v4_l1(row + 16 * c + 8);
+        } else {
+          u[j][0] = u[j][1] = make_uint4(0, 0, 0, 0);
+        }
       }
 #pragma unroll
       for (int j = 0; j < kQuantUnroll; ++j) {
-        const int v = v0 + 32 * j;
-        if (v - lane >= vpr) break;  // warp-uniform
-        float f[8];
-        bf16x8_to_f32(u[j], f);
+        const int c = c0 + 32 * j;
+        if (c >= bpr) break;
+        float f[16];
+        bf16x16_to_f32(u[j][0], u[j][1], f);
         uint32_t sfc;
-        const uint32_t packed = nvfp4_vector(f, g, six_g, sfc);
-        if (v < vpr) {
-          crow[v] = packed;
-          if ((v & 1) == 0) sf[sf_offset(r, v >> 1, c4)] = static_cast<uint8_t>(sfc);
-        }
+        crow[c] = nvfp4_block16(f, g, six_g, sfc);
+        sf_row[(c >> 2) * 512 + (c & 3)] = static_cast<uint8_t>(sfc);
       }
     }
   }
@@ -327,29 +360,6 @@ __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
                : "r"(addr));
   return r;
 }
-
-// One 16-element block held by one lane: the same arithmetic as
-// nvfp4_vector, with the block-level steps done once per block.  Returns the
-// 16 E2M1 codes (element 2i in the low nibble of byte i); sfc receives the
-// block's E4M3 scale code.
-__device__ __forceinline__ uint2 nvfp4_block16(float (&f)[16], float g, float six_g,
-                                               uint32_t& sfc) {
-  float bmax = fabsf(f[0]);
-#pragma unroll
-  for (int i = 1; i < 16; ++i) bmax = fmaxf(bmax, fabsf(f[i]));
-  sfc = cvt_e4m3x2(bmax / six_g, 0.0f) & 0xFFu;
-  const float s = e4m3_value(sfc) * g;
-  const float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
-  float lo[8], hi[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    lo[i] = f[i] * inv;
-    hi[i] = f[8 + i] * inv;
-  }
-  return make_uint2(cvt_e2m1x8(lo), cvt_e2m1x8(hi));
-}
-
-constexpr unsigned long long kKeyMask = 0xFFFFFFFF00000000ull;
 
 // Bounded spin until the word's upper half equals `key`; its lower half out.
 __device__ __forceinline__ bool spin_for_key(const unsigned long long* p, unsigned long long key,
@@ -472,14 +482,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     // this row's scale bytes: 512-byte tile (r / 128, c / 4), byte (r % 32) * 16 + (r / 32 % 4) * 4 + c % 4
     uint8_t* sf_row = sf + static_cast<int64_t>(r >> 7) * c4 * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
     for (int c = lane; c < bpr; c += 32) {
-      const uint4 u0 = lds_v4(row + 32u * c), u1 = lds_v4(row + 32u * c + 16u);
-      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
       float f[16];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        f[2 * j] = __uint_as_float(w[j] << 16);
-        f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-      }
+      bf16x16_to_f32(lds_v4(row + 32u * c), lds_v4(row + 32u * c + 16u), f);
       uint32_t sfc;
       crow[c] = nvfp4_block16(f, g, six_g, sfc);
       sf_row[(c >> 2) * 512 + (c & 3)] = static_cast<uint8_t>(sfc);
