@@ -84,10 +84,8 @@ struct PairCfg {
   static constexpr int EPI_COLS = BN / 2;   // accumulator columns per epilogue warp
   static constexpr int EPI_SUB = 32;        // staging sub-tile: 32 rows x 32 columns (64-byte rows)
   static constexpr int EPI_BYTES = EPI_WARPS * 32 * EPI_SUB * 2;
-  // registers: launched with 65536 / 512 = 128 per thread, then rebalanced.
-  // Keep the margins: with 72 for the scale writers (ptxas reported no
-  // spills) repeated launches produced wrong scales in whole 32-row slices,
-  // i.e. a writer warp lost register contents to the epilogue's increase.
+  // registers: launched with 65536 / 512 = 128 per thread, then rebalanced so
+  // that an epilogue thread holds its 128 accumulator columns at once
   static constexpr int REGS_CTRL = 56, REGS_SFW = 80, REGS_EPI = 184;
   static constexpr int BAR_BYTES = 512;
   static constexpr int STAGES_FIT =
@@ -383,8 +381,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
                        : "=r"(vb[4 * i]), "=r"(vb[4 * i + 1]), "=r"(vb[4 * i + 2]), "=r"(vb[4 * i + 3])
                        : "r"(slot + C::SFA_BYTES + (cb * C::SF_CHUNKS + jb) * 512 + lane * 16));
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sf_empty_bar(r));  // slot read: the loader may refill it
         // set n is free once the MMAs of stage g - S have completed; the full
         // barrier of that stage has completed too, so the arrival below counts
         // towards stage g
@@ -409,7 +405,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(leader_full0 + 8u * n);
+        // The slot goes back to the loader only now that the stores have
+        // consumed every value read from it.  Released right after the
+        // ld.shared instructions, the refill (the stage R later) could land
+        // before the warp's last loads had read the slot: a few lanes then
+        // stored that stage's B scales for the last MMA of the stage.
+        if (lane == 0) {
+          mbar_arrive_remote(leader_full0 + 8u * n);
+          mbar_arrive(sf_empty_bar(r));
+        }
         if (++r == R) { r = 0; rph ^= 1u; }
         if (++n == S) { n = 0; nph ^= 1u; }
       }

@@ -1,10 +1,14 @@
-"""Repeated runs of one layer with many tiles per CTA pair: every run within
-the oracle's tolerance on sampled rows, and runs differing from each other by
-at most one bf16 rounding step (the two MMA issuers' later stages may reach
-the tensor pipe in either order, which can move an fp32 sum by an ulp and a
-bf16 output by one step, never more).  A race between the issuers, the
-accumulator and the epilogue shows up here as larger or out-of-tolerance
-differences in a few tiles of some runs."""
+"""Repeated back-to-back runs of one layer with many tiles per CTA pair.
+
+Every run must equal the first within one bf16 rounding step per output (the
+GEMM issues each accumulator's MMAs in a fixed order, so runs are expected to
+be identical; one step of slack keeps the test about correctness rather than
+bit-reproducibility), and the first run plus every row where any run
+differs must be within the oracle's tolerance.  Forty launches without a
+synchronisation in between: a race between the scale loader and the scale
+writers (a shared-memory slot refilled before a warp's last loads had read
+it) corrupted the last MMA of a stage in a few lanes about once in a hundred
+launches of the 16384-row layer while single runs passed."""
 
 import numpy as np
 import pytest
@@ -18,8 +22,26 @@ import fp8_gemm_diffusion_b200 as mxq
 
 pytestmark = pytest.mark.gpu
 
+RUNS = 40
 
-@pytest.mark.parametrize("fmt,M,K,N", [("nvfp4", 4608, 3072, 21504), ("mxfp8", 4608, 3072, 9216)])
+
+def _oracle(fmt, A, W, b, rows):
+    sel = torch.as_tensor(rows)
+    if fmt == "nvfp4":
+        qa = Q.quantize_nvfp4(A[sel], global_amax=Q.amax(A))
+        qw = Q.quantize_nvfp4(W)
+        Ad = Q.dequant_nvfp4(qa["codes"], qa["sf"], qa["g"])
+        Wd = Q.dequant_nvfp4(qw["codes"], qw["sf"], qw["g"])
+    else:
+        qa = Q.quantize_mxfp8(A[sel])
+        qw = Q.quantize_mxfp8(W)
+        Ad = Q.dequant_mxfp8(qa["codes"], qa["sf"])
+        Wd = Q.dequant_mxfp8(qw["codes"], qw["sf"])
+    return G.linear_ref(Ad, Wd, b)
+
+
+@pytest.mark.parametrize("fmt,M,K,N", [("nvfp4", 4608, 3072, 12288), ("nvfp4", 16384, 3072, 12288),
+                                       ("mxfp8", 4608, 3072, 9216)])
 def test_repeated_runs(fmt, M, K, N):
     g = torch.Generator().manual_seed(77 + N)
     W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
@@ -27,27 +49,26 @@ def test_repeated_runs(fmt, M, K, N):
     A = torch.randn(M, K, generator=g).to(torch.bfloat16)
     layer = mxq.Weight(W.to(DEV), b.to(DEV), fmt=fmt)
     Ad = A.to(DEV)
-    ys = [mxq.linear_forward(layer, Ad, min_dim=1) for _ in range(4)]
+    y0 = mxq.linear_forward(layer, Ad, min_dim=1)
+    y0f = y0.float()
+    bad_rows = set()
+    worst = []
+    for i in range(1, RUNS):
+        y = mxq.linear_forward(layer, Ad, min_dim=1)  # no synchronisation between launches
+        d = (y.float() - y0f).abs()
+        bound = torch.maximum(y.float().abs(), y0f.abs()) * 2.0 ** -7 + 1e-6
+        over = d > bound
+        if bool(over.any()):
+            idx = over.nonzero()
+            worst.append((i, int(idx.shape[0]), idx[:3].tolist()))
+        diff_rows = (d > 0).any(dim=1).nonzero().flatten().tolist()
+        bad_rows.update(diff_rows[:16])
+        del y, d, bound, over
     torch.cuda.synchronize()
     assert mxq.get_device_error() == mxq.OK
-    y0 = ys[0].float()
-    for y in ys[1:]:
-        d = (y.float() - y0).abs()
-        bound = torch.maximum(y.float().abs(), y0.abs()) * 2.0 ** -7 + 1e-6
-        bad = (d > bound).nonzero()
-        assert bad.numel() == 0, f"runs differ by more than a bf16 step at {bad[:4].tolist()}"
+    assert not worst, f"runs differ from run 0 by more than a bf16 step: {worst[:4]}"
     rng = np.random.default_rng(M + N)
-    rows = np.unique(np.concatenate([np.arange(0, 8), np.arange(M - 8, M), rng.integers(0, M, 48)]))
-    if fmt == "nvfp4":
-        qa = Q.quantize_nvfp4(A[torch.as_tensor(rows)], global_amax=Q.amax(A))
-        qw = Q.quantize_nvfp4(W)
-        Ad_ = Q.dequant_nvfp4(qa["codes"], qa["sf"], qa["g"])
-        Wd = Q.dequant_nvfp4(qw["codes"], qw["sf"], qw["g"])
-    else:
-        qa = Q.quantize_mxfp8(A[torch.as_tensor(rows)])
-        qw = Q.quantize_mxfp8(W)
-        Ad_ = Q.dequant_mxfp8(qa["codes"], qa["sf"])
-        Wd = Q.dequant_mxfp8(qw["codes"], qw["sf"])
-    Y, T = G.linear_ref(Ad_, Wd, b)
-    for k, y in enumerate(ys):
-        assert_within_tol(y[torch.as_tensor(rows, device=DEV)], Y, T, f"{fmt} run {k}")
+    rows = np.unique(np.concatenate([np.arange(0, 8), np.arange(M - 8, M), rng.integers(0, M, 48),
+                                     np.array(sorted(bad_rows)[:64], dtype=np.int64)]))
+    Y, T = _oracle(fmt, A, W, b, rows)
+    assert_within_tol(y0[torch.as_tensor(rows, device=DEV)], Y, T, f"{fmt} {M}x{K}x{N} run 0")
