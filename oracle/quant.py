@@ -27,6 +27,9 @@ NVFP4, tensor X [R, K]:
   3. s = value(sf) * g;  inv = 1 / s, or 0 when s == 0.
   4. code_i = E2M1(x_i * inv).  Element 2j goes in the low nibble of byte j.
   5. Dequantised value = value(code) * value(sf) * g.
+  Without the per-tensor scale (the listing's flag switched off; reading: the
+  block scale then carries the whole range) g = 1 in every step above, so
+  sf = E4M3(bamax / 6), saturating at 448, and no amax is taken.
 
 MXFP8, tensor X [R, K] (OCP MX v1.0, scale from floor(log2 amax)):
   1. per row and 32-element block: e = floor(log2(bamax)), exact;
@@ -138,20 +141,27 @@ def unpack_fp4(packed: np.ndarray) -> np.ndarray:
     return out
 
 
-def quantize_nvfp4(x, global_amax=None):
+def quantize_nvfp4(x, global_amax=None, tensor_scale=True):
     """NVFP4 quantisation of X [R, K] (K a multiple of 16).
 
     Returns dict(codes=[R, K/2] uint8 packed, sf=[R, K/16] uint8 (E4M3),
     sf_swz=flat swizzled scale array, g=float32 per-tensor scale,
     amax=float32).  ``global_amax`` overrides the tensor's own amax (used when
     the amax comes from elsewhere, e.g. a reduction across shards).
+    ``tensor_scale=False``: no per-tensor scale, g = 1 and no amax is taken
+    (amax is reported as 0).
     """
     x = _as_f32(x)
     R, K = x.shape
     if K % NVFP4_BLOCK:
         raise ValueError("K must be a multiple of 16")
-    a = amax(x) if global_amax is None else _F32(global_amax)
-    g = nvfp4_global_scale(a)
+    if tensor_scale:
+        a = amax(x) if global_amax is None else _F32(global_amax)
+        g = nvfp4_global_scale(a)
+    else:
+        if global_amax is not None:
+            raise ValueError("global_amax needs the per-tensor scale")
+        a, g = _F32(0.0), _F32(1.0)
     blocks = x.reshape(R, K // NVFP4_BLOCK, NVFP4_BLOCK)
     bamax = np.max(np.abs(blocks), axis=2) if K else np.zeros((R, 0), _F32)
     denom = _F32(_F32(6.0) * g)

@@ -74,6 +74,63 @@ def test_nvfp4_exact_blocks_reproduce(j):
     assert np.array_equal(deq, X.astype(np.float64))
 
 
+def test_nvfp4_without_tensor_scale_exact_blocks():
+    # g = 1: blocks c_i * e (e an E4M3 value, one |c_i| = 6) give sf = e and
+    # codes c_i, so the dequantised tensor is the input, bit for bit
+    rng = np.random.default_rng(7)
+    e2 = F.e2m1_decode(np.arange(16))
+    e4 = F.e4m3_decode(np.arange(1, 0x7F))
+    R, K = 6, 96
+    codes = rng.integers(0, 16, size=(R, K))
+    scales = rng.choice(e4[e4 >= 2.0 ** -6], size=(R, K // 16))
+    X = np.zeros((R, K))
+    for r in range(R):
+        for b in range(K // 16):
+            cs = codes[r, b * 16:(b + 1) * 16]
+            cs[rng.integers(0, 16)] = rng.choice([7, 15])
+            X[r, b * 16:(b + 1) * 16] = e2[cs] * scales[r, b]
+    X = X.astype(np.float32)
+    xb = _bf16(X)
+    assert np.array_equal(xb.float().numpy(), X), "fixture values must be bf16-exact"
+    q = Q.quantize_nvfp4(xb, tensor_scale=False)
+    assert q["g"] == f32(1.0) and q["amax"] == f32(0.0)
+    assert np.array_equal(F.e4m3_decode(q["sf"]), scales)
+    assert np.array_equal(Q.dequant_nvfp4(q["codes"], q["sf"], q["g"]), X.astype(np.float64))
+
+
+def test_nvfp4_without_tensor_scale_saturation_and_underflow():
+    x = np.zeros((3, 16), dtype=np.float32)
+    # bamax / 6 = 1024 > 448: the scale saturates at 448 (0x7E); then
+    # 6144 / 448 = 13.7 saturates to +6, -700 / 448 = -1.5625 rounds to -1.5,
+    # 448 / 448 = 1
+    x[0, 0], x[0, 1], x[0, 2] = 6144.0, -700.0, 448.0
+    # bamax / 6 = 2^-10: half of E4M3's smallest subnormal 2^-9, a tie -> 0,
+    # so the block's scale and codes are 0
+    x[1, 0] = 6 * 2.0 ** -10
+    # bamax / 6 = 3 * 2^-10: a tie between 2^-9 (code 1) and 2^-8 (code 2) -> 2^-8
+    x[2, 0] = 6 * 3 * 2.0 ** -10
+    q = Q.quantize_nvfp4(x, tensor_scale=False)
+    assert list(q["sf"][:, 0]) == [0x7E, 0x00, 0x02]
+    c = Q.unpack_fp4(q["codes"])
+    assert list(c[0, :3]) == [0x7, 0xB, 0x2]          # +6, -1.5, +1
+    assert np.all(c[1] == 0)
+    # row 2: x / 2^-8 = 4.5 -> E2M1 tie between 4 and 6 -> 4 (even mantissa)
+    assert c[2, 0] == 0x6
+
+
+def test_nvfp4_without_tensor_scale_is_unit_g():
+    # g = amax / 2688 is exactly 1 for amax = 2688, so the variant equals the
+    # general recipe with that amax
+    x = torch.randn(40, 128, generator=torch.Generator().manual_seed(12)) * 5
+    x[3, 7] = 9000.0
+    a = Q.quantize_nvfp4(x.bfloat16(), tensor_scale=False)
+    b = Q.quantize_nvfp4(x.bfloat16(), global_amax=np.float32(2688.0))
+    assert b["g"] == f32(1.0)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["sf"], b["sf"])
+    with pytest.raises(ValueError):
+        Q.quantize_nvfp4(x, global_amax=1.0, tensor_scale=False)
+
+
 @pytest.mark.parametrize("k", [-20, -5, 0, 7])
 def test_mxfp8_exact_blocks_reproduce(k):
     rng = np.random.default_rng(100 + k)
