@@ -41,6 +41,9 @@ NVFP4 = 1
 MXFP8 = 2
 BF16 = 3
 FORMATS = {"nvfp4": NVFP4, "mxfp8": MXFP8, "bf16": BF16}
+# mxq_weight_prepare flags (mxq_weight.flags)
+WEIGHT_KEEP_BF16 = 1
+WEIGHT_NO_TENSOR_SCALE = 2
 
 _i64 = ctypes.c_int64
 _ptr = ctypes.c_void_p
@@ -51,7 +54,7 @@ _int = ctypes.c_int
 class mxq_weight(ctypes.Structure):
     _fields_ = [
         ("format", ctypes.c_int32),
-        ("keep_bf16", ctypes.c_int32),
+        ("flags", ctypes.c_int32),
         ("N", _i64),
         ("K", _i64),
         ("w_bf16", _ptr),
@@ -191,6 +194,7 @@ def amax(x, amax_out, rows=None, k=None, ld=None, stream=None) -> None:
 
 
 def quantize_nvfp4(x, amax_in, codes, sf, g_out, rows=None, k=None, ld=None, stream=None) -> None:
+    """amax_in=None: NVFP4 without a per-tensor scale (g = 1)."""
     rows, k, ld = _shape2(x, rows, k, ld)
     _check(_quantize_nvfp4(_addr(x), rows, k, ld, _addr(amax_in), _addr(codes), _addr(sf),
                            _addr(g_out), _stream(stream)), "mxq_quantize_nvfp4")
@@ -214,9 +218,10 @@ def weight_storage_bytes(N: int, K: int, fmt) -> int:
     return _weight_storage_bytes(N, K, _fmt(fmt))
 
 
-def weight_prepare(fmt, w, N, K, bias, keep_bf16, storage, storage_bytes, stream=None) -> mxq_weight:
+def weight_prepare(fmt, w, N, K, bias, flags, storage, storage_bytes, stream=None) -> mxq_weight:
+    """flags: WEIGHT_KEEP_BF16 | WEIGHT_NO_TENSOR_SCALE bits (0: the defaults)."""
     out = mxq_weight()
-    _check(_weight_prepare(_fmt(fmt), _addr(w), N, K, _addr(bias), int(bool(keep_bf16)),
+    _check(_weight_prepare(_fmt(fmt), _addr(w), N, K, _addr(bias), int(flags),
                            _addr(storage), storage_bytes, ctypes.byref(out), _stream(stream)),
            "mxq_weight_prepare")
     return out
@@ -274,14 +279,17 @@ class Weight:
     into (kept alive here).  Allocation is torch's; quantisation runs in
     mxq_weight_prepare."""
 
-    def __init__(self, w, bias=None, fmt="nvfp4", keep_bf16=False, stream=None):
+    def __init__(self, w, bias=None, fmt="nvfp4", keep_bf16=False, tensor_scale=True, stream=None):
+        """tensor_scale=False: NVFP4 without a per-tensor scale (g = 1 for the
+        weight and every activation)."""
         import torch
         N, K = w.shape
         self.w, self.bias, self.fmt = w, bias, _fmt(fmt)
+        flags = (WEIGHT_KEEP_BF16 if keep_bf16 else 0) | (0 if tensor_scale else WEIGHT_NO_TENSOR_SCALE)
         nbytes = weight_storage_bytes(N, K, self.fmt) if not keep_bf16 else 0
         self.storage = (torch.empty(max(nbytes, 256), dtype=torch.uint8, device=w.device)
                         if nbytes else None)
-        self.handle = weight_prepare(self.fmt, w, N, K, bias, keep_bf16, self.storage, nbytes,
+        self.handle = weight_prepare(self.fmt, w, N, K, bias, flags, self.storage, nbytes,
                                      stream=stream)
 
     @property

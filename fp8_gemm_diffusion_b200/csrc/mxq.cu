@@ -461,7 +461,7 @@ const char* mxq_status_string(mxq_status s) {
   return "unknown status";
 }
 
-int mxq_version(void) { return (1 << 16) | 0; }
+int mxq_version(void) { return (1 << 16) | 1; }
 
 int mxq_last_cuda_error(void) { return t_last_cuda_error; }
 
@@ -497,7 +497,7 @@ mxq_status mxq_quantize_nvfp4(const void* x_bf16, int64_t rows, int64_t k, int64
                               float* g_dev, mxq_stream_t stream) {
   mxq_status st = check_bf16_matrix(x_bf16, rows, k, ld);
   if (st != MXQ_OK) return st;
-  if (amax_dev == nullptr || g_dev == nullptr) return MXQ_ERR_INVALID_ARG;
+  if (g_dev == nullptr) return MXQ_ERR_INVALID_ARG;
   if (rows > 0 && k > 0 && (codes == nullptr || sf_swz == nullptr)) return MXQ_ERR_INVALID_ARG;
   if (k % 64 != 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(codes) || !aligned16(sf_swz)) return MXQ_ERR_ALIGNMENT;
@@ -506,8 +506,9 @@ mxq_status mxq_quantize_nvfp4(const void* x_bf16, int64_t rows, int64_t k, int64
   int dev, sms;
   if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
   if (rows == 0 || k == 0) return MXQ_OK;
-  return launch_quant_nvfp4(x_bf16, rows, k, ld, amax_dev, 1, codes, sf_swz, g_dev, nullptr,
-                            reinterpret_cast<cudaStream_t>(stream), sms);
+  // no amax: the kernel reduces zero values to amax 0, whose scale is g = 1
+  return launch_quant_nvfp4(x_bf16, rows, k, ld, amax_dev, amax_dev != nullptr ? 1 : 0, codes,
+                            sf_swz, g_dev, nullptr, reinterpret_cast<cudaStream_t>(stream), sms);
 }
 
 mxq_status mxq_quantize_mxfp8(const void* x_bf16, int64_t rows, int64_t k, int64_t ld,
@@ -563,16 +564,20 @@ size_t mxq_weight_storage_bytes(int64_t N, int64_t K, mxq_format f) {
 }
 
 mxq_status mxq_weight_prepare(mxq_format f, const void* w_bf16, int64_t N, int64_t K,
-                              const void* bias_bf16, int keep_bf16, void* storage,
+                              const void* bias_bf16, int flags, void* storage,
                               size_t storage_bytes, mxq_weight* out, mxq_stream_t stream) {
   if (out == nullptr || !valid_format(f)) return MXQ_ERR_INVALID_ARG;
+  if (flags & ~(MXQ_WEIGHT_KEEP_BF16 | MXQ_WEIGHT_NO_TENSOR_SCALE)) return MXQ_ERR_INVALID_ARG;
+  const bool keep_bf16 = (flags & MXQ_WEIGHT_KEEP_BF16) != 0;
+  const bool no_tensor_scale = (flags & MXQ_WEIGHT_NO_TENSOR_SCALE) != 0;
+  if (no_tensor_scale && f != MXQ_NVFP4) return MXQ_ERR_INVALID_ARG;
   mxq_status st = check_bf16_matrix(w_bf16, N, K, K);
   if (st != MXQ_OK) return st;
   if (bias_bf16 != nullptr && (reinterpret_cast<uintptr_t>(bias_bf16) & 1u)) return MXQ_ERR_ALIGNMENT;
   mxq_weight w;
   std::memset(&w, 0, sizeof(w));
   w.format = f;
-  w.keep_bf16 = keep_bf16 ? 1 : 0;
+  w.flags = flags;
   w.N = N;
   w.K = K;
   w.w_bf16 = w_bf16;
@@ -593,7 +598,15 @@ mxq_status mxq_weight_prepare(mxq_format f, const void* w_bf16, int64_t N, int64
     int dev, sms;
     if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (f == MXQ_NVFP4) {
+    if (f == MXQ_NVFP4 && no_tensor_scale) {
+      // g_W = 1: the quantiser reduces no amax values (amax 0 -> g = 1) and
+      // writes 0 to the amax slot
+      if (N > 0 && K > 0 &&
+          (st = launch_quant_nvfp4(w_bf16, N, K, K, nullptr, 0, codes, sf, g, amax, s, sms)) != MXQ_OK)
+        return st;
+      w.g_dev = g;
+      w.amax_dev = amax;
+    } else if (f == MXQ_NVFP4) {
       if ((st = launch_amax(w_bf16, N, K, K, amax, s, sms)) != MXQ_OK) return st;
       if (N > 0 && K > 0 &&
           (st = launch_quant_nvfp4(w_bf16, N, K, K, amax, 1, codes, sf, g, nullptr, s, sms)) != MXQ_OK)
@@ -614,7 +627,7 @@ mxq_status mxq_weight_prepare(mxq_format f, const void* w_bf16, int64_t N, int64
 int mxq_linear_path(const mxq_weight* w, int64_t M, const mxq_linear_opts* opts) {
   if (w == nullptr) return 0;
   const int64_t min_dim = (opts != nullptr && opts->min_dim > 0) ? opts->min_dim : 1024;
-  if (w->keep_bf16 || w->format == MXQ_BF16) return MXQ_BF16;
+  if ((w->flags & MXQ_WEIGHT_KEEP_BF16) || w->format == MXQ_BF16) return MXQ_BF16;
   int64_t m = M < w->K ? M : w->K;
   m = m < w->N ? m : w->N;
   if (m < min_dim) return MXQ_BF16;
@@ -670,7 +683,11 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
   float* g = reinterpret_cast<float*>(base + 4);
   uint8_t* codes = base + l.codes_off;
   uint8_t* sf = base + l.sf_off;
-  if (f == MXQ_NVFP4) {
+  if (f == MXQ_NVFP4 && (w->flags & MXQ_WEIGHT_NO_TENSOR_SCALE)) {
+    // no per-tensor scale: one pass, g = 1 (no amax values to reduce)
+    if ((st = launch_quant_nvfp4(x_bf16, M, K, K, nullptr, 0, codes, sf, g, amax, s, sms)) != MXQ_OK)
+      return st;
+  } else if (f == MXQ_NVFP4) {
     float* partials = reinterpret_cast<float*>(base + kPartialsOff);
     const FusedPlan plan = plan_fused(M, K, sms);
     if (plan.grid > 0) {
@@ -704,7 +721,7 @@ int mxq_linear_kernel_count(const mxq_weight* w, int64_t M, const mxq_linear_opt
   if (w == nullptr || M <= 0 || w->N <= 0) return 0;
   const int path = mxq_linear_path(w, M, opts);
   if (path == MXQ_BF16) return 1;
-  if (path == MXQ_MXFP8) return 2;
+  if (path == MXQ_MXFP8 || (w->flags & MXQ_WEIGHT_NO_TENSOR_SCALE)) return 2;
   int dev, sms;
   if (current_device(&dev, &sms) != MXQ_OK) return -1;
   return plan_fused(M, w->K, sms).grid > 0 ? 2 : 3;

@@ -110,11 +110,13 @@ mxq_status mxq_amax(const void* x_bf16, int64_t rows, int64_t k, int64_t ld,
  *   saturating, sign kept.
  * Inputs: x_bf16 [rows][ld]; amax_dev: fp32 amax of the tensor (device),
  *   usually from mxq_amax (it may be any amax the caller chooses, e.g. a
- *   reduction over shards).
+ *   reduction over shards).  amax_dev == NULL selects NVFP4 without a
+ *   per-tensor scale (the listing's use_dynamic_per_tensor_scale switched
+ *   off): g = 1, so sf = E4M3(bamax / 6), saturating at 448.
  * Outputs: codes [rows][k/2] bytes (mxq_codes_bytes), sf_swz
  *   (mxq_sf_bytes bytes, padding written as 0), *g_dev.
  * Errors: k % 64 != 0 -> UNSUPPORTED_SHAPE (whole 4-column scale tiles);
- *   NULL pointers, misalignment as above.
+ *   NULL x / codes / sf_swz / g_dev, misalignment as above.
  */
 mxq_status mxq_quantize_nvfp4(const void* x_bf16, int64_t rows, int64_t k, int64_t ld,
                               const float* amax_dev, uint8_t* codes, uint8_t* sf_swz,
@@ -162,16 +164,24 @@ mxq_status mxq_gemm_blockscaled(mxq_format f, int64_t M, int64_t N, int64_t K,
  * by mxq_weight_prepare; the caller owns every buffer it points to and must
  * keep w_bf16, bias_bf16 and the storage alive while the handle is used.
  */
+/* Flags of mxq_weight_prepare and mxq_weight.flags. */
+enum {
+  MXQ_WEIGHT_KEEP_BF16 = 1,       /* always run this layer as a bf16 GEMM          */
+  MXQ_WEIGHT_NO_TENSOR_SCALE = 2  /* NVFP4 without a per-tensor scale: g = 1 for
+                                     both W and every activation (no amax pass)    */
+};
+
 typedef struct mxq_weight {
   int32_t format;         /* mxq_format the weight is quantised to           */
-  int32_t keep_bf16;      /* 1: always run this layer as a bf16 GEMM         */
+  int32_t flags;          /* MXQ_WEIGHT_* bits                               */
   int64_t N, K;           /* W is [N, K]                                     */
   const void* w_bf16;     /* original bf16 weights [N][K] (row stride K)     */
   const void* bias_bf16;  /* [N] bf16 or NULL                                */
   const uint8_t* codes;   /* quantised codes inside the storage (or NULL)    */
   const uint8_t* sf;      /* swizzled scales inside the storage (or NULL)    */
   const float* g_dev;     /* NVFP4 per-tensor scale g_W (device) or NULL     */
-  const float* amax_dev;  /* amax of W (device) or NULL                      */
+  const float* amax_dev;  /* amax of W (device; 0 without a per-tensor scale)
+                             or NULL                                         */
 } mxq_weight;
 
 /* Device bytes mxq_weight_prepare needs for format f (0 for MXQ_BF16). */
@@ -182,11 +192,14 @@ size_t mxq_weight_storage_bytes(int64_t N, int64_t K, mxq_format f);
  * weights ahead of time in the same format as the activations, "...NVFP4
  * Weight" in its TorchAO config name).  Runs mxq_amax + mxq_quantize_* on W
  * into `storage` (mxq_weight_storage_bytes bytes, 256-byte aligned) and fills
- * *out.  With keep_bf16 != 0 or f == MXQ_BF16 nothing is quantised (storage
- * may be NULL) and the layer always runs in bf16.
+ * *out.  flags: MXQ_WEIGHT_* bits (0 = the defaults; other bits ->
+ * INVALID_ARG).  With MXQ_WEIGHT_KEEP_BF16 or f == MXQ_BF16 nothing is
+ * quantised (storage may be NULL) and the layer always runs in bf16.  With
+ * MXQ_WEIGHT_NO_TENSOR_SCALE (NVFP4 only, else INVALID_ARG) W is quantised
+ * with g_W = 1 and mxq_linear quantises activations with g = 1 (no amax).
  */
 mxq_status mxq_weight_prepare(mxq_format f, const void* w_bf16, int64_t N, int64_t K,
-                              const void* bias_bf16, int keep_bf16, void* storage,
+                              const void* bias_bf16, int flags, void* storage,
                               size_t storage_bytes, mxq_weight* out, mxq_stream_t stream);
 
 /* Options of mxq_linear.  A NULL pointer means the defaults. */
@@ -201,7 +214,8 @@ typedef struct mxq_linear_opts {
 
 /*
  * mxq_linear_path - the format mxq_linear would run for M rows: MXQ_BF16
- * when w->keep_bf16, when w->format is MXQ_BF16, or when min(M, K, N) <
+ * when w->flags has MXQ_WEIGHT_KEEP_BF16, when w->format is MXQ_BF16, or when
+ * min(M, K, N) <
  * min_dim (article, "Detailed by section": selective quantisation, layers
  * too small to gain, or accuracy-sensitive embeddings, stay in bf16);
  * w->format otherwise.  Pure host function.  Returns 0 for a NULL w.
@@ -224,7 +238,9 @@ size_t mxq_linear_workspace_bytes(int64_t M, int64_t K, mxq_format f);
  * quantised by one cooperative kernel (amax and quantisation in one pass
  * over HBM, the amax exchanged through a bounded grid barrier whose state
  * lives in the workspace); larger ones by two kernels (partial maxima, then
- * quantisation).  Calls sharing one workspace must be ordered on the GPU.
+ * quantisation).  A weight prepared with MXQ_WEIGHT_NO_TENSOR_SCALE takes
+ * no amax: one quantisation kernel with g = 1, then the GEMM (alpha = 1).
+ * Calls sharing one workspace must be ordered on the GPU.
  */
 mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* y_bf16,
                       void* ws, size_t ws_bytes, const mxq_linear_opts* opts,
@@ -263,7 +279,8 @@ mxq_status mxq_linear_noalloc(const mxq_weight* w, const void* x_bf16, int64_t M
 /*
  * mxq_linear_kernel_count - how many kernels one mxq_linear call with these
  * arguments launches on the current device: 1 (bf16 GEMM), 2 (MXFP8
- * quantise + GEMM, or single-pass NVFP4 quantise + GEMM) or 3 (NVFP4 partial
+ * quantise + GEMM, single-pass NVFP4 quantise + GEMM, or NVFP4 without a
+ * per-tensor scale: quantise + GEMM) or 3 (NVFP4 partial
  * maxima + quantise + GEMM); 0 when M or N is 0 (nothing is launched) or w
  * is NULL; -1 when the current device cannot be queried.  Uses the same
  * decisions as mxq_linear.  No GPU work.

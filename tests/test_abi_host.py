@@ -67,7 +67,11 @@ def _st(fn, *a):
 def test_quantize_rejects_bad_arguments():
     q = lambda *a, **kw: mxq.quantize_nvfp4(*a, **kw)
     assert _st(q, None, A16, A16, A16, A16, 4, 64, 64) == mxq.ERR_INVALID_ARG
-    assert _st(q, A16, None, A16, A16, A16, 4, 64, 64) == mxq.ERR_INVALID_ARG
+    assert _st(q, A16, A16, A16, A16, None, 4, 64, 64) == mxq.ERR_INVALID_ARG  # g_out
+    if not torch.cuda.is_available():
+        # a NULL amax selects g = 1 (no per-tensor scale): past the argument
+        # checks, stopped only by the missing device
+        assert _st(q, A16, None, A16, A16, A16, 4, 64, 64) == mxq.ERR_ARCH
     assert _st(q, A16 + 2, A16, A16, A16, A16, 4, 64, 64) == mxq.ERR_ALIGNMENT
     assert _st(q, A16, A16, A16 + 8, A16, A16, 4, 64, 64) == mxq.ERR_ALIGNMENT
     assert _st(q, A16, A16, A16, A16, A16, 4, 48, 48) == mxq.ERR_UNSUPPORTED_SHAPE
@@ -96,7 +100,7 @@ def test_gemm_rejects_bad_arguments():
 
 
 def test_workspace_and_storage_checks():
-    w = mxq.mxq_weight(format=mxq.NVFP4, keep_bf16=0, N=4096, K=4096, w_bf16=A16, bias_bf16=None,
+    w = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=4096, K=4096, w_bf16=A16, bias_bf16=None,
                        codes=A16, sf=A16, g_dev=A16, amax_dev=A16)
     need = mxq.linear_workspace_bytes(4096, 4096, "nvfp4")
     assert _st(mxq.linear, w, A16, 4096, A16, A16, need - 1) == mxq.ERR_WORKSPACE
@@ -122,28 +126,48 @@ def test_valid_call_without_gpu_fails_loudly():
 def test_linear_path_follows_selection_rule():
     for B in (1, 4):
         for l in workloads.flux_linear_stack(batch=B):
-            w = mxq.mxq_weight(format=mxq.NVFP4, keep_bf16=0, N=l["N"], K=l["K"])
+            w = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=l["N"], K=l["K"])
             want = mxq.BF16 if D.use_bf16(l["M"], l["K"], l["N"]) else mxq.NVFP4
             assert mxq.linear_path(w, l["M"]) == want, l
-    w = mxq.mxq_weight(format=mxq.MXFP8, keep_bf16=0, N=1024, K=1024)
+    w = mxq.mxq_weight(format=mxq.MXFP8, flags=0, N=1024, K=1024)
     assert mxq.linear_path(w, 1024) == mxq.MXFP8
     assert mxq.linear_path(w, 1023) == mxq.BF16
     assert mxq.linear_path(w, 1024, min_dim=2048) == mxq.BF16
-    w.keep_bf16 = 1
+    w.flags = mxq.WEIGHT_KEEP_BF16
     assert mxq.linear_path(w, 8192) == mxq.BF16
 
 
 def test_linear_kernel_count_host_cases():
-    w = mxq.mxq_weight(format=mxq.MXFP8, keep_bf16=0, N=1024, K=1024)
+    w = mxq.mxq_weight(format=mxq.MXFP8, flags=0, N=1024, K=1024)
     assert mxq.linear_kernel_count(w, 0) == 0            # nothing launched
     assert mxq.linear_kernel_count(w, 1023) == 1         # bf16 GEMM
     assert mxq.linear_kernel_count(w, 1024) == 2         # MXFP8 quantise + GEMM
-    w = mxq.mxq_weight(format=mxq.NVFP4, keep_bf16=0, N=0, K=1024)
+    w = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=0, K=1024)
     assert mxq.linear_kernel_count(w, 4096) == 0
     if not torch.cuda.is_available():
         # the NVFP4 choice (one or two quantiser kernels) depends on the SM count
-        w = mxq.mxq_weight(format=mxq.NVFP4, keep_bf16=0, N=1024, K=1024)
+        w = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=1024, K=1024)
         assert mxq.linear_kernel_count(w, 4096) == -1
+
+
+def test_no_tensor_scale_weight_host_cases():
+    # NVFP4 without a per-tensor scale: no amax pass, one quantiser + the GEMM,
+    # decided without querying the device
+    w = mxq.mxq_weight(format=mxq.NVFP4, flags=mxq.WEIGHT_NO_TENSOR_SCALE, N=1024, K=1024)
+    assert mxq.linear_path(w, 4096) == mxq.NVFP4
+    assert mxq.linear_kernel_count(w, 4096) == 2
+    assert mxq.linear_kernel_count(w, 1023) == 1         # still bf16 below the threshold
+    w.flags |= mxq.WEIGHT_KEEP_BF16
+    assert mxq.linear_path(w, 4096) == mxq.BF16
+
+
+def test_weight_prepare_rejects_bad_flags():
+    out = mxq.mxq_weight()
+    # unknown bits, and the no-tensor-scale bit on a format without a per-tensor scale
+    for fmt, flags in ((mxq.NVFP4, 4), (mxq.NVFP4, 1 << 20), (mxq.MXFP8, mxq.WEIGHT_NO_TENSOR_SCALE),
+                       (mxq.BF16, mxq.WEIGHT_NO_TENSOR_SCALE)):
+        st = mxq._weight_prepare(fmt, A16, 1024, 1024, None, flags, None, 0, mxq.ctypes.byref(out), None)
+        assert st == mxq.ERR_INVALID_ARG, (fmt, flags, st)
 
 
 class _FakeEvent:
@@ -154,7 +178,7 @@ class _FakeEvent:
 
 
 def test_linear_rejects_half_an_event_pair():
-    w = mxq.mxq_weight(format=mxq.NVFP4, keep_bf16=0, N=4096, K=4096, w_bf16=A16, bias_bf16=None,
+    w = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=4096, K=4096, w_bf16=A16, bias_bf16=None,
                        codes=A16, sf=A16, g_dev=A16, amax_dev=A16)
     need = mxq.linear_workspace_bytes(4096, 4096, "nvfp4")
     half = (_FakeEvent(0x1000), _FakeEvent(0))

@@ -57,7 +57,7 @@ def test_noalloc_bf16_path_and_size_limit():
     assert G.within_tol(y.float().cpu().numpy(), ref.float().cpu().numpy(), T).all()
     # a quantised layer whose workspace exceeds the static scratch is refused
     # before anything is enqueued
-    big = mxq.mxq_weight(format=mxq.NVFP4, keep_bf16=0, N=3072, K=12288, w_bf16=1 << 20,
+    big = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=3072, K=12288, w_bf16=1 << 20,
                          codes=1 << 20, sf=1 << 20, g_dev=1 << 20)
     M_big = 16896
     assert mxq.linear_workspace_bytes(M_big, 12288, "nvfp4") > mxq.NOALLOC_SCRATCH_BYTES
