@@ -13,6 +13,9 @@ Plain numpy, written to be checked by eye against the definitions:
 * ``quant``    - NVFP4 and MXFP8 quantisation, scale-factor layout.
 * ``gemm``     - float64 reference of the quantised linear and its tolerance.
 * ``dispatch`` - the selective-quantisation rule.
+* ``producer`` - a linear layer with the GELU activation fused into its
+  epilogue, and that epilogue's error scale (the oracle of the fused-producer
+  kernel that comes next; no GPU kernel uses it yet).
 
 Every function is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle_*.py`` to facts other than itself (code tables, tie cases,
@@ -22,7 +25,7 @@ checked only indirectly, through GEMM parity on the GPU (parity unpinned on
 the CPU side).
 """
 
-from . import formats, quant, gemm, dispatch  # noqa: F401
+from . import formats, quant, gemm, dispatch, producer  # noqa: F401
 from .formats import *  # noqa: F401,F403
 from .quant import *  # noqa: F401,F403
 from .gemm import *  # noqa: F401,F403
