@@ -378,6 +378,9 @@ def run_gpu(args, rank, world, local_rank):
             "value": round(bf16_tflops, 2), "unit": UNIT,
             "ms_per_step": round(bf16_ms, 5),
             "speedup_of_value": round(value / bf16_tflops, 3),
+            "fraction_of_dense_peak": {"nominal": round(bf16_tflops / 2250.0, 4),
+                                       "nominal_peak_tflops": 2250.0,
+                                       "measured_burst": round(bf16_tflops / peaks["bf16"], 4)},
         },
         "clocks": sampler.summary(),
         "e2e": e2e,
