@@ -183,3 +183,33 @@ def test_linear_rejects_half_an_event_pair():
     need = mxq.linear_workspace_bytes(4096, 4096, "nvfp4")
     half = (_FakeEvent(0x1000), _FakeEvent(0))
     assert _st(mxq.linear, w, A16, 4096, A16, A16, need, None, None, half) == mxq.ERR_INVALID_ARG
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes mirrors of mxq_weight and mxq_linear_opts have the C header's
+    size and field offsets (a mismatch would hand the library shifted fields)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    fields = {"mxq_weight": [f[0] for f in mxq.mxq_weight._fields_],
+              "mxq_linear_opts": [f[0] for f in mxq.mxq_linear_opts._fields_]}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "mxq.h"', "int main(void) {"]
+    for st, names in fields.items():
+        lines.append(f'  printf("{st} size %zu\\n", sizeof({st}));')
+        for n in names:
+            lines.append(f'  printf("{st} {n} %zu\\n", offsetof({st}, {n}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-I", os.path.join(root, "include"), str(src), "-o", str(exe)],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {tuple(l.split()[:2]): int(l.split()[2]) for l in out if l.strip()}
+    for st, cls in (("mxq_weight", mxq.mxq_weight), ("mxq_linear_opts", mxq.mxq_linear_opts)):
+        assert got[(st, "size")] == ctypes.sizeof(cls), st
+        for n in fields[st]:
+            assert got[(st, n)] == getattr(cls, n).offset, (st, n)
