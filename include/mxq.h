@@ -159,11 +159,6 @@ mxq_status mxq_gemm_blockscaled(mxq_format f, int64_t M, int64_t N, int64_t K,
 
 /* ----------------------------------------------------- weights / linear -- */
 
-/*
- * A prepared linear layer.  Plain data: device pointers plus sizes.  Filled
- * by mxq_weight_prepare; the caller owns every buffer it points to and must
- * keep w_bf16, bias_bf16 and the storage alive while the handle is used.
- */
 /* Flags of mxq_weight_prepare and mxq_weight.flags. */
 enum {
   MXQ_WEIGHT_KEEP_BF16 = 1,       /* always run this layer as a bf16 GEMM          */
@@ -171,6 +166,11 @@ enum {
                                      both W and every activation (no amax pass)    */
 };
 
+/*
+ * A prepared linear layer.  Plain data: device pointers plus sizes.  Filled
+ * by mxq_weight_prepare; the caller owns every buffer it points to and must
+ * keep w_bf16, bias_bf16 and the storage alive while the handle is used.
+ */
 typedef struct mxq_weight {
   int32_t format;         /* mxq_format the weight is quantised to           */
   int32_t flags;          /* MXQ_WEIGHT_* bits                               */
