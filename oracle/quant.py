@@ -180,12 +180,19 @@ def _floor_log2(a: np.ndarray) -> np.ndarray:
     return e.astype(np.int64) - 1
 
 
-def quantize_mxfp8(x):
+def quantize_mxfp8(x, scale_rule="floor"):
     """MXFP8 quantisation of X [R, K] (K a multiple of 32).
 
     Returns dict(codes=[R, K] uint8 (E4M3), sf=[R, K/32] uint8 (E8M0),
     sf_swz=flat swizzled scale array).
+
+    scale_rule "floor" is the OCP rule above.  "rceil" (TorchAO's ceiling
+    mode; the pages name only the OCP standard) takes the smallest X with
+    bamax <= 448 * 2^X, so no element saturates; since 2^e <= bamax < 2^(e+1)
+    that X is e - 8 or e - 7, decided by one exact comparison.
     """
+    if scale_rule not in ("floor", "rceil"):
+        raise ValueError(scale_rule)
     x = _as_f32(x)
     R, K = x.shape
     if K % MXFP8_BLOCK:
@@ -194,7 +201,11 @@ def quantize_mxfp8(x):
     bamax = np.max(np.abs(blocks), axis=2) if K else np.zeros((R, 0), _F32)
     pos = bamax > 0
     e = np.where(pos, _floor_log2(np.where(pos, bamax, _F32(1.0))), -(1 << 20))
-    X = np.clip(e - 8, -127, 127)
+    X = e - 8
+    if scale_rule == "rceil":
+        over = bamax.astype(np.float64) > 448.0 * np.ldexp(1.0, np.maximum(X, -1000))
+        X = np.where(pos & over, X + 1, X)
+    X = np.clip(X, -127, 127)
     sf = (X + 127).astype(np.uint8)
     mult = np.ldexp(np.ones_like(X, dtype=np.float64), -X).astype(_F32)  # 2^-X, exact in fp32
     q = (blocks * mult[:, :, None]).astype(_F32)

@@ -235,3 +235,33 @@ def test_pack_unpack_fp4():
     p = Q.pack_fp4(c)
     assert p[0, 0] == (c[0, 0] | (c[0, 1] << 4))
     assert np.array_equal(Q.unpack_fp4(p), c)
+
+
+def test_mxfp8_rceil_scale_closed_form():
+    # one element per block, |x| = 2^p * (1 + f): the ceiling rule adds one to
+    # the floor rule's exponent exactly when 1 + f > 448 / 256 = 1.75
+    for p in range(-120, 120, 9):
+        for f in (0.0, 0.5, 0.75, 0.7578125, 0.99):
+            x = np.zeros((1, 32), dtype=np.float32)
+            x[0, 5] = f32(2.0 ** p * (1 + f))
+            qf = Q.quantize_mxfp8(x)
+            qc = Q.quantize_mxfp8(x, scale_rule="rceil")
+            want = max(p - 8 + (1 if 1 + f > 1.75 else 0), -127) + 127
+            assert qc["sf"][0, 0] == want, (p, f)
+            assert qf["sf"][0, 0] == max(p - 8, -127) + 127
+
+
+def test_mxfp8_rceil_never_saturates():
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal((64, 256)) * np.exp(rng.uniform(-20, 20, size=(64, 1)))).astype(np.float32)
+    q = Q.quantize_mxfp8(x, scale_rule="rceil")
+    X = q["sf"].astype(np.int64) - 127
+    bamax = np.abs(x).reshape(64, 8, 32).max(axis=2).astype(np.float64)
+    scaled = bamax * np.ldexp(1.0, -X)
+    # the block maximum lands in the top binade (224, 448] and so encodes
+    # without saturating
+    assert np.all((scaled > 224) & (scaled <= 448))
+    deq = Q.dequant_mxfp8(q["codes"], q["sf"])
+    assert np.all(np.abs(deq).reshape(64, 8, 32).max(axis=2) <= 448.0 * np.ldexp(1.0, X))
+    with pytest.raises(ValueError):
+        Q.quantize_mxfp8(x, scale_rule="ceil")
