@@ -176,7 +176,9 @@ def run_gpu(args, rank, world, local_rank):
     # one prepared weight, then per-set copies of everything a step touches
     W = case.W.to(dev)
     bias = case.bias.to(dev) if case.bias is not None else None
-    base_w = mxq.Weight(W, bias, fmt=fmt)
+    # NVFP4 without a per-tensor scale (g = 1, no amax pass) on request
+    unit_g = fmt == "nvfp4" and args.no_tensor_scale
+    base_w = mxq.Weight(W, bias, fmt=fmt, tensor_scale=not unit_g)
     ws_bytes = mxq.linear_workspace_bytes(M, K, fmt)
     per_set = M * K * 2 + mxq.weight_storage_bytes(N, K, fmt) + M * N * 2 + ws_bytes
     nsets = max(2, int(np.ceil(3 * L2_BYTES / per_set)))
@@ -342,7 +344,8 @@ def run_gpu(args, rank, world, local_rank):
         "data": "synthetic (seeded, FLUX-shaped; random-init weights)",
         "config": {
             "workload": case.name, "format": fmt, "M": M, "K": K, "N": N,
-            "bias": case.bias is not None, "parallelism": f"replicas x{world}",
+            "bias": case.bias is not None, "per_tensor_scale": not unit_g,
+            "parallelism": f"replicas x{world}",
             "step": "mxq_linear: activation amax + quantisation + block-scaled GEMM (weights pre-quantised)",
             "l2": f"rotating {nsets} buffer sets ({nsets * per_set / 2**20:.0f} MiB > 126 MiB L2)",
         },
@@ -660,6 +663,8 @@ def main():
                     help="M,K,N of a seeded random layer instead of a named workload (profiling)")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp8"], help="format for --shape")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-tensor-scale", action="store_true",
+                    help="NVFP4 without a per-tensor scale (g = 1 for weight and activation)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
