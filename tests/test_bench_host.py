@@ -1,0 +1,58 @@
+"""Host-side parts of bench.py that need no GPU: the reference arm's JSON
+line (the oracle timed on the host cores, bounded), the clock summary and the
+peak denominators."""
+
+import json
+import os
+import subprocess
+import sys
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(*args):
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT,
+                         capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1, out.stdout
+    return json.loads(lines[0])
+
+
+def test_reference_arm_line():
+    d = _run("--impl", "reference", "--steps", "1", "--warmup", "3", "--workload", "c1")
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["value"] > 0 and d["higher_is_better"] is True
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"] == "c1_nvfp4_256x1024x1024"
+
+
+def test_reference_arm_for_the_stack_is_unavailable():
+    d = _run("--impl", "reference", "--workload", "c5")
+    assert d["impl"] == "reference" and "unavailable" in d
+
+
+def test_clock_summary_flags_throttling():
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s._h, s.max_mhz = object(), 1965
+    s.samples = [1800, 1900, 1965]
+    s.reasons = 0x4 | 0x1  # sw_power_cap, and gpu_idle which is not reported
+    out = s.summary()
+    assert out == {"sm_mhz": 1900.0, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"], "samples": 3}
+    s._h = None
+    assert s.summary()["reasons"] == ["unavailable"]
+
+
+def test_peaks_come_from_the_measured_file_or_the_fallback():
+    p = bench._peaks()
+    assert p["source"] in ("measured", "fallback")
+    assert p["bf16"] > 0 and p["bf16_sustained"] > 0 and p["hbm"] > 0
+    assert bench.whole_job_tflops(2, 10, 1e12, 1000.0) == 20.0
