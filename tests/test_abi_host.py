@@ -53,7 +53,24 @@ def test_sizes_match_oracle_layout(rows, k):
     assert ws >= 256 + rows * k // 2 + Q.sf_bytes(rows, k, 16) and ws % 256 == 0
 
 
-A16 = 1 << 20  # a 16-byte aligned fake device address (never dereferenced)
+_KEEP = []
+
+
+def dev(nbytes: int, misalign: int = 0) -> int:
+    """A device address for a buffer of `nbytes` (plus `misalign` bytes of offset).
+
+    On a machine with a GPU this is a real allocation of that size, so that a
+    call which got past its host checks by mistake could only touch valid
+    memory.  Without a GPU every call returns before any launch, and a fixed
+    256-byte aligned address stands in (nothing dereferences it there)."""
+    if torch.cuda.is_available():
+        t = torch.zeros(int(nbytes) + 256, dtype=torch.uint8, device="cuda")
+        _KEEP.append(t)
+        return t.data_ptr() + misalign
+    return (1 << 20) + misalign
+
+
+SMALL = 1 << 16  # covers every buffer of the small shapes below (4 x 64, 128 x 128 x 256)
 
 
 def _st(fn, *a):
@@ -66,50 +83,54 @@ def _st(fn, *a):
 
 def test_quantize_rejects_bad_arguments():
     q = lambda *a, **kw: mxq.quantize_nvfp4(*a, **kw)
-    assert _st(q, None, A16, A16, A16, A16, 4, 64, 64) == mxq.ERR_INVALID_ARG
-    assert _st(q, A16, A16, A16, A16, None, 4, 64, 64) == mxq.ERR_INVALID_ARG  # g_out
+    assert _st(q, None, dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), 4, 64, 64) == mxq.ERR_INVALID_ARG
+    assert _st(q, dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), None, 4, 64, 64) == mxq.ERR_INVALID_ARG  # g_out
     if not torch.cuda.is_available():
         # a NULL amax selects g = 1 (no per-tensor scale): past the argument
         # checks, stopped only by the missing device
-        assert _st(q, A16, None, A16, A16, A16, 4, 64, 64) == mxq.ERR_ARCH
-    assert _st(q, A16 + 2, A16, A16, A16, A16, 4, 64, 64) == mxq.ERR_ALIGNMENT
-    assert _st(q, A16, A16, A16 + 8, A16, A16, 4, 64, 64) == mxq.ERR_ALIGNMENT
-    assert _st(q, A16, A16, A16, A16, A16, 4, 48, 48) == mxq.ERR_UNSUPPORTED_SHAPE
-    assert _st(q, A16, A16, A16, A16, A16, 4, 64, 60) == mxq.ERR_INVALID_ARG  # ld < k
-    assert _st(q, A16, A16, A16, A16, A16, 4, 64, 68) == mxq.ERR_ALIGNMENT  # ld % 8
-    assert _st(q, A16, A16, A16, A16, A16, -1, 64, 64) == mxq.ERR_INVALID_ARG
+        assert _st(q, dev(SMALL), None, dev(SMALL), dev(SMALL), dev(SMALL), 4, 64, 64) == mxq.ERR_ARCH
+    assert _st(q, dev(SMALL, 2), dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), 4, 64, 64) == mxq.ERR_ALIGNMENT
+    assert _st(q, dev(SMALL), dev(SMALL), dev(SMALL, 8), dev(SMALL), dev(SMALL), 4, 64, 64) == mxq.ERR_ALIGNMENT
+    assert _st(q, dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), 4, 48, 48) == mxq.ERR_UNSUPPORTED_SHAPE
+    assert _st(q, dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), 4, 64, 60) == mxq.ERR_INVALID_ARG  # ld < k
+    assert _st(q, dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), 4, 64, 68) == mxq.ERR_ALIGNMENT  # ld % 8
+    assert _st(q, dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), -1, 64, 64) == mxq.ERR_INVALID_ARG
     m = lambda *a, **kw: mxq.quantize_mxfp8(*a, **kw)
-    assert _st(m, A16, A16, A16, 4, 64, 64) == mxq.ERR_UNSUPPORTED_SHAPE  # k % 128
-    assert _st(m, A16, None, A16, 4, 128, 128) == mxq.ERR_INVALID_ARG
+    assert _st(m, dev(SMALL), dev(SMALL), dev(SMALL), 4, 64, 64) == mxq.ERR_UNSUPPORTED_SHAPE  # k % 128
+    assert _st(m, dev(SMALL), None, dev(SMALL), 4, 128, 128) == mxq.ERR_INVALID_ARG
 
 
 def test_gemm_rejects_bad_arguments():
     g = lambda *a: mxq.gemm_blockscaled(*a)
-    ok = ("nvfp4", 128, 128, 256, A16, A16, A16, A16, A16, A16, None, A16, 128)
+    ok = ("nvfp4", 128, 128, 256, dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), dev(SMALL), None, dev(SMALL), 128)
     assert _st(g, 9, *ok[1:]) == mxq.ERR_INVALID_ARG
     assert _st(g, "nvfp4", 128, 128, 96, *ok[4:]) == mxq.ERR_UNSUPPORTED_SHAPE
     assert _st(g, "mxfp8", 128, 128, 192, *ok[4:]) == mxq.ERR_UNSUPPORTED_SHAPE
     assert _st(g, "nvfp4", 128, 128, 0, *ok[4:]) == mxq.ERR_UNSUPPORTED_SHAPE
     assert _st(g, *ok[:4], None, *ok[5:]) == mxq.ERR_INVALID_ARG
     assert _st(g, *ok[:6], None, *ok[7:]) == mxq.ERR_INVALID_ARG  # NVFP4 needs g_A
-    assert _st(g, *ok[:11], A16 + 16, 120) == mxq.ERR_INVALID_ARG  # ldy < N
-    assert _st(g, *ok[:11], A16, 132) == mxq.ERR_ALIGNMENT
-    assert _st(g, *ok[:11], A16 + 4, 128) == mxq.ERR_ALIGNMENT
-    assert _st(g, "bf16", 128, 128, 12, A16, None, None, A16, None, None, None, A16, 128) \
+    assert _st(g, *ok[:11], dev(SMALL, 16), 120) == mxq.ERR_INVALID_ARG  # ldy < N
+    assert _st(g, *ok[:11], dev(SMALL), 132) == mxq.ERR_ALIGNMENT
+    assert _st(g, *ok[:11], dev(SMALL, 4), 128) == mxq.ERR_ALIGNMENT
+    assert _st(g, "bf16", 128, 128, 12, dev(SMALL), None, None, dev(SMALL), None, None, None, dev(SMALL), 128) \
         == mxq.ERR_UNSUPPORTED_SHAPE
 
 
 def test_workspace_and_storage_checks():
-    w = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=4096, K=4096, w_bf16=A16, bias_bf16=None,
-                       codes=A16, sf=A16, g_dev=A16, amax_dev=A16)
-    need = mxq.linear_workspace_bytes(4096, 4096, "nvfp4")
-    assert _st(mxq.linear, w, A16, 4096, A16, A16, need - 1) == mxq.ERR_WORKSPACE
-    assert _st(mxq.linear, w, A16, 4096, A16, A16 + 16, need) == mxq.ERR_ALIGNMENT
-    assert _st(mxq.linear, w, A16, 4096, A16, None, need) == mxq.ERR_INVALID_ARG
-    need_w = mxq.weight_storage_bytes(4096, 4096, "mxfp8")
-    assert _st(mxq.weight_prepare, "mxfp8", A16, 4096, 4096, None, 0, A16, need_w - 1) \
+    N = K = M = 4096
+    need = mxq.linear_workspace_bytes(M, K, "nvfp4")
+    w = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=N, K=K, w_bf16=dev(N * K * 2), bias_bf16=None,
+                       codes=dev(N * K // 2), sf=dev(mxq.sf_bytes(N, K, "nvfp4")), g_dev=dev(4),
+                       amax_dev=dev(4))
+    x, y, ws = dev(M * K * 2), dev(M * N * 2), dev(need + 16)
+    assert _st(mxq.linear, w, x, M, y, ws, need - 1) == mxq.ERR_WORKSPACE
+    assert _st(mxq.linear, w, x, M, y, ws + 16, need) == mxq.ERR_ALIGNMENT
+    assert _st(mxq.linear, w, x, M, y, None, need) == mxq.ERR_INVALID_ARG
+    need_w = mxq.weight_storage_bytes(N, K, "mxfp8")
+    storage = dev(need_w)
+    assert _st(mxq.weight_prepare, "mxfp8", w.w_bf16, N, K, None, 0, storage, need_w - 1) \
         == mxq.ERR_WORKSPACE
-    assert _st(mxq.weight_prepare, "mxfp8", A16, 4096, 4000, None, 0, A16, 1 << 30) \
+    assert _st(mxq.weight_prepare, "mxfp8", w.w_bf16, N, 4000, None, 0, storage, need_w) \
         == mxq.ERR_UNSUPPORTED_SHAPE
 
 
@@ -117,9 +138,9 @@ def test_workspace_and_storage_checks():
 def test_valid_call_without_gpu_fails_loudly():
     # no CPU fallback: a well-formed call on a machine without an sm_100 GPU
     # returns MXQ_ERR_ARCH and computes nothing
-    assert _st(mxq.quantize_mxfp8, A16, A16, A16, 4, 128, 128) == mxq.ERR_ARCH
-    assert _st(mxq.gemm_blockscaled, "bf16", 8, 8, 64, A16, None, None, A16, None, None, None,
-               A16, 8) == mxq.ERR_ARCH
+    assert _st(mxq.quantize_mxfp8, dev(SMALL), dev(SMALL), dev(SMALL), 4, 128, 128) == mxq.ERR_ARCH
+    assert _st(mxq.gemm_blockscaled, "bf16", 8, 8, 64, dev(SMALL), None, None, dev(SMALL), None, None, None,
+               dev(SMALL), 8) == mxq.ERR_ARCH
     assert mxq.get_device_error() == mxq.ERR_ARCH
 
 
@@ -163,10 +184,11 @@ def test_no_tensor_scale_weight_host_cases():
 
 def test_weight_prepare_rejects_bad_flags():
     out = mxq.mxq_weight()
+    w16 = dev(1024 * 1024 * 2)
     # unknown bits, and the no-tensor-scale bit on a format without a per-tensor scale
     for fmt, flags in ((mxq.NVFP4, 4), (mxq.NVFP4, 1 << 20), (mxq.MXFP8, mxq.WEIGHT_NO_TENSOR_SCALE),
                        (mxq.BF16, mxq.WEIGHT_NO_TENSOR_SCALE)):
-        st = mxq._weight_prepare(fmt, A16, 1024, 1024, None, flags, None, 0, mxq.ctypes.byref(out), None)
+        st = mxq._weight_prepare(fmt, w16, 1024, 1024, None, flags, None, 0, mxq.ctypes.byref(out), None)
         assert st == mxq.ERR_INVALID_ARG, (fmt, flags, st)
 
 
@@ -178,11 +200,19 @@ class _FakeEvent:
 
 
 def test_linear_rejects_half_an_event_pair():
-    w = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=4096, K=4096, w_bf16=A16, bias_bf16=None,
-                       codes=A16, sf=A16, g_dev=A16, amax_dev=A16)
-    need = mxq.linear_workspace_bytes(4096, 4096, "nvfp4")
-    half = (_FakeEvent(0x1000), _FakeEvent(0))
-    assert _st(mxq.linear, w, A16, 4096, A16, A16, need, None, None, half) == mxq.ERR_INVALID_ARG
+    N = K = M = 4096
+    w = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=N, K=K, w_bf16=dev(N * K * 2), bias_bf16=None,
+                       codes=dev(N * K // 2), sf=dev(mxq.sf_bytes(N, K, "nvfp4")), g_dev=dev(4),
+                       amax_dev=dev(4))
+    need = mxq.linear_workspace_bytes(M, K, "nvfp4")
+    if torch.cuda.is_available():
+        real = torch.cuda.Event(enable_timing=True)
+        real.record()  # torch creates the event's handle on its first record
+        half = (real, _FakeEvent(0))
+    else:
+        half = (_FakeEvent(0x1000), _FakeEvent(0))
+    assert _st(mxq.linear, w, dev(M * K * 2), M, dev(M * N * 2), dev(need), need, None, None, half) \
+        == mxq.ERR_INVALID_ARG
 
 
 def test_struct_layouts_match_the_header(tmp_path):

@@ -14,7 +14,7 @@ import torch
 
 from oracle import formats as F
 from oracle import quant as Q
-from tests._golden import keyed
+from tests._golden import _lines, keyed
 
 f32 = np.float32
 
@@ -218,6 +218,40 @@ def test_nvfp4_error_bound():
     s = F.e4m3_decode(q["sf"]) * float(q["g"])
     err = np.abs(deq - x.float().numpy()).reshape(16, 16, 16)
     assert np.all(err <= s[:, :, None] * 1.0 + 1e-12)
+
+
+def _sf_layout_fixture():
+    """(r, c, C, offset) entries and (rows, C, size) entries of sf_layout.txt."""
+    entries, sizes = [], []
+    for parts in _lines("sf_layout.txt"):
+        if parts[0] == "size":
+            sizes.append(tuple(int(v) for v in parts[1:4]))
+        else:
+            entries.append(tuple(int(v) for v in parts[:4]))
+    return entries, sizes
+
+
+def test_swizzle_matches_hand_worked_layout():
+    # each scale alone in an otherwise empty matrix must land at the byte the
+    # published layout gives (a swapped or dropped term moves it)
+    entries, sizes = _sf_layout_fixture()
+    assert len(entries) >= 12
+    for r, c, C, off in entries:
+        R = r + 1
+        sf = np.zeros((R, C), dtype=np.uint8)
+        sf[r, c] = 0xA5
+        swz = Q.swizzle_sf(sf)
+        assert swz.size == Q.sf_bytes(R, C * 16, 16)
+        assert np.flatnonzero(swz).tolist() == [off], (r, c, C, off, np.flatnonzero(swz))
+        # and the inverse reads the byte at that offset back to (r, c)
+        flat = np.zeros(swz.size, dtype=np.uint8)
+        flat[off] = 0x5A
+        back = Q.unswizzle_sf(flat, R, C)
+        assert back[r, c] == 0x5A and np.count_nonzero(back) == 1, (r, c, C, off)
+    for rows, C, size in sizes:
+        assert Q.sf_bytes(rows, C * 16, 16) == size
+        assert Q.sf_bytes(rows, C * 32, 32) == size
+        assert Q.swizzle_sf(np.ones((rows, C), dtype=np.uint8)).size == size
 
 
 def test_swizzle_roundtrip_and_padding():
