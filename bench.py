@@ -50,6 +50,10 @@ import workloads  # noqa: E402
 METRIC = "block-scaled GEMM TFLOPS incl. act quant; % of dense FP4/FP8 peak"
 UNIT = "TFLOP/s"
 L2_BYTES = 126 * 1024 * 1024
+# GPU spin ahead of each timed region (cycles; ~0.5 ms): the host gets ahead
+SPIN_CYCLES = 1_000_000
+# a GEMM timed inside a region at least this long is held to the sustained peak
+SUSTAINED_MIN_MS = 1000.0
 # Dense tensor peaks (TFLOP/s) for the roofline: the measured cuBLAS bf16
 # figure of this machine pool times the nominal FP4:BF16 (4x) / FP8:BF16 (2x)
 # ratio of B200; fallback numbers when no measurement file is present.
@@ -87,7 +91,11 @@ def _nvml_id(local_rank: int):
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while running."""
+    """Samples SM clock and throttle reasons through NVML while running.
+
+    Every sample carries a host timestamp, so that a caller can count the
+    samples that fell inside a given window (``mark``) as well as those of
+    the whole measurement."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -95,10 +103,10 @@ class ClockSampler:
         0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device, period_s: float = 0.002):
+    def __init__(self, device, period_s: float = 0.0002):
         self.period = period_s
-        self.samples = []
-        self.reasons = 0
+        self.samples = []  # (host time, SM MHz, reason bits)
+        self.windows = {}
         self.max_mhz = None
         self._stop = threading.Event()
         self._thread = None
@@ -113,12 +121,15 @@ class ClockSampler:
         except Exception:
             self._h = None
 
-    def _run(self):
+    def _sample(self):
         nv = self._nv
+        self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM),
+                             nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)))
+
+    def _run(self):
         while not self._stop.is_set():
             try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self._sample()
             except Exception:
                 break
             time.sleep(self.period)
@@ -128,17 +139,40 @@ class ClockSampler:
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
 
+    def mark(self, name, t0, t1):
+        """Record [t0, t1] (host perf_counter times) as a named window."""
+        self.windows[name] = (t0, t1)
+
     def stop(self):
         if self._thread is not None:
             self._stop.set()
             self._thread.join()
 
-    def summary(self):
+    def _summ(self, samples):
+        mhz = [m for _, m, _ in samples]
+        bits = 0
+        for _, _, r in samples:
+            bits |= r
+        names = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(mhz)) if mhz else None, "reasons": names,
+                "samples": len(mhz), "sm_mhz_min": min(mhz) if mhz else None}
+
+    def summary(self, window=None):
+        """Median SM clock and the reasons seen, over all samples, with the
+        counts inside each marked window (``window`` picks the headline one)."""
         if self._h is None or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
-        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": names, "samples": len(self.samples)}
+        out = self._summ(self.samples)
+        out["sm_max_mhz"] = self.max_mhz
+        out["period_ms"] = self.period * 1e3
+        out["windows"] = {}
+        for name, (t0, t1) in self.windows.items():
+            out["windows"][name] = self._summ([x for x in self.samples if t0 <= x[0] <= t1])
+        if window in self.windows and out["windows"][window]["samples"]:
+            w = out["windows"][window]
+            out["sm_mhz_headline"] = w["sm_mhz"]
+            out["samples_headline"] = w["samples"]
+        return out
 
 
 # ------------------------------------------------------- rank aggregation
@@ -212,10 +246,18 @@ def run_gpu(args, rank, world, local_rank):
     quantize_public(A0)
     torch.cuda.synchronize()
 
+    # The path the dispatcher takes for this layer.  C1 is the NVFP4 W4A4
+    # single-GEMM configuration: its 256 x 1024 x 1024 shape is below the
+    # selective rule's 1024 threshold, so it is run with min_dim = 1 to time
+    # the NVFP4 path it names (the line reports the path actually taken).
+    min_dim = args.min_dim if args.min_dim is not None else (1 if case.name.startswith("c1") else None)
+    path = mxq.linear_path(base_w.handle, M, min_dim)
+    run_fmt = {mxq.NVFP4: "nvfp4", mxq.MXFP8: "mxfp8", mxq.BF16: "bf16"}[path]
+
     def step(i, gemm_events=None):
         st = sets[i % nsets]
         mxq.linear(st["w"], st["x"], M, st["y"], st["ws"], ws_bytes, stream=stream,
-                   gemm_events=gemm_events)
+                   gemm_events=gemm_events, min_dim=min_dim)
 
     def gemm_only(i):
         st = sets[i % nsets]
@@ -225,7 +267,7 @@ def run_gpu(args, rank, world, local_rank):
                              stream=stream)
 
     # kernels one mxq_linear call launches here (the library's own dispatch decision)
-    launches_per_step = mxq.linear_kernel_count(base_w.handle, M)
+    launches_per_step = mxq.linear_kernel_count(base_w.handle, M, min_dim)
     assert launches_per_step > 0, launches_per_step
     dist = world > 1
     if dist:
@@ -245,21 +287,31 @@ def run_gpu(args, rank, world, local_rank):
         b.record(stream)
     torch.cuda.synchronize()
     sampler = ClockSampler(_nvml_id(local_rank))
-    if dist:
-        tdist.barrier()
-    torch.cuda.synchronize()
     sampler.start()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for i in range(args.steps):
-        step(args.warmup + i)
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    sampler.stop()
-    if dist:
-        tdist.barrier()
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
+
+    def timed_pass(name, n, fn):
+        """n calls of fn(i) between two events; max over ranks of the span.
+        A short spin kernel ahead of the start event lets the host enqueue the
+        first steps before the GPU reaches them, so the span holds GPU work
+        only (no launch gap at its start)."""
+        if dist:
+            tdist.barrier()
+        torch.cuda.synchronize()
+        torch.cuda._sleep(SPIN_CYCLES)
+        t_start.record(stream)
+        h0 = time.perf_counter()
+        for i in range(n):
+            fn(i)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        sampler.mark(name, h0, time.perf_counter())
+        if dist:
+            tdist.barrier()
+        return max_over_ranks(t_start.elapsed_time(t_end), dev)
+
+    total_ms = timed_pass("headline", args.steps, lambda i: step(args.warmup + i))
     if mxq.get_device_error() != mxq.OK:
         raise RuntimeError("device-side timeout during the timed steps")
 
@@ -267,17 +319,7 @@ def run_gpu(args, rank, world, local_rank):
     # launch: the GEMM's average duration inside the steps (the roofline's
     # kernel).  An event recorded between two kernels costs the next one its
     # programmatic early launch, so the headline value comes from the first pass.
-    if dist:
-        tdist.barrier()
-    torch.cuda.synchronize()
-    t_start.record(stream)
-    for i in range(args.steps):
-        step(args.warmup + i, gemm_evs[i])
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    if dist:
-        tdist.barrier()
-    total_ev_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
+    total_ev_ms = timed_pass("gemm_events", args.steps, lambda i: step(args.warmup + i, gemm_evs[i]))
     gemm_ms = float(np.mean([a.elapsed_time(b) for a, b in gemm_evs]))
     if mxq.get_device_error() != mxq.OK:
         raise RuntimeError("device-side timeout during the timed steps")
@@ -285,15 +327,8 @@ def run_gpu(args, rank, world, local_rank):
     # the same step with one buffer set only (inputs stay in L2 between steps):
     # the hot number beside the L2-cold headline
     hot_steps = max(10, min(args.steps, 500))
-    if dist:
-        tdist.barrier()
-    torch.cuda.synchronize()
-    t_start.record(stream)
-    for _ in range(hot_steps):
-        step(0)
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    hot_ms = max_over_ranks(t_start.elapsed_time(t_end), dev) / hot_steps
+    hot_ms = timed_pass("hot", hot_steps, lambda i: step(0)) / hot_steps
+    sampler.stop()
 
     # for comparison: the GEMM launched alone, back to back, same stream
     reps = max(10, min(args.steps, 50))
@@ -319,15 +354,27 @@ def run_gpu(args, rank, world, local_rank):
     e2e = run_e2e(mxq, case, base_w, dev, stream, args, dist)
 
     peaks = _peaks()
-    # timed inside a long run of steps: the sustained peak (burst reported beside it)
-    peak = peaks["bf16_sustained"] * NOMINAL_RATIO[fmt]
-    peak_burst = peaks["bf16"] * NOMINAL_RATIO[fmt]
+    # The denominator follows the timed region's length: the burst figure
+    # (cuBLAS timed alone) unless the GEMM ran inside a region of at least a
+    # second, long enough for the power cap to settle the clock (the sustained
+    # figure).  The other one is reported beside it.
+    sustained = total_ev_ms >= SUSTAINED_MIN_MS
+    peak_burst = peaks["bf16"] * NOMINAL_RATIO[run_fmt]
+    peak_sus = peaks["bf16_sustained"] * NOMINAL_RATIO[run_fmt]
+    peak = peak_sus if sustained else peak_burst
     achieved = flops / (gemm_ms * 1e-3) / 1e12
+    clocks = sampler.summary("headline")
+    gemm_mhz = (clocks.get("windows", {}).get("gemm_events", {}) or {}).get("sm_mhz")
     value = whole_job_tflops(world, args.steps, flops, total_ms)
     bf16_tflops = whole_job_tflops(world, 1, flops, bf16_ms)
     step_ms = total_ms / args.steps
-    qbytes = M * K * 2 + mxq.codes_bytes(M, K, fmt) + mxq.sf_bytes(M, K, fmt)
-    nominal = {"nvfp4": 9000.0, "mxfp8": 4500.0}[fmt]
+    qbytes = M * K * 2 + mxq.codes_bytes(M, K, run_fmt) + mxq.sf_bytes(M, K, run_fmt)
+    nominal = {"nvfp4": 9000.0, "mxfp8": 4500.0, "bf16": 2250.0}[run_fmt]
+    step_text = {"nvfp4": "mxq_linear: activation amax + NVFP4 quantisation + block-scaled GEMM "
+                          "(weights pre-quantised)",
+                 "mxfp8": "mxq_linear: MXFP8 activation quantisation + block-scaled GEMM "
+                          "(weights pre-quantised)",
+                 "bf16": "mxq_linear: bf16 GEMM (selective rule)"}[run_fmt]
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -339,14 +386,16 @@ def run_gpu(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e2m1+e4m3 (nvfp4), fp32 accumulate, bf16 out" if fmt == "nvfp4"
-        else "e4m3+e8m0 (mxfp8), fp32 accumulate, bf16 out",
+        "dtype": {"nvfp4": "e2m1+e4m3 (nvfp4), fp32 accumulate, bf16 out",
+                  "mxfp8": "e4m3+e8m0 (mxfp8), fp32 accumulate, bf16 out",
+                  "bf16": "bf16, fp32 accumulate, bf16 out"}[run_fmt],
         "data": "synthetic (seeded, FLUX-shaped; random-init weights)",
         "config": {
-            "workload": case.name, "format": fmt, "M": M, "K": K, "N": N,
+            "workload": case.name, "format": fmt, "path": run_fmt,
+            "min_dim": min_dim if min_dim is not None else 1024, "M": M, "K": K, "N": N,
             "bias": case.bias is not None, "per_tensor_scale": not unit_g,
             "parallelism": f"replicas x{world}",
-            "step": "mxq_linear: activation amax + quantisation + block-scaled GEMM (weights pre-quantised)",
+            "step": step_text,
             "l2": f"rotating {nsets} buffer sets ({nsets * per_set / 2**20:.0f} MiB > 126 MiB L2)",
         },
         "fraction_of_dense_peak": {"nominal": round(value / nominal, 4), "nominal_peak_tflops": nominal},
@@ -362,17 +411,25 @@ def run_gpu(args, rank, world, local_rank):
                 "ms_per_step": round(hot_ms, 5), "steps": hot_steps,
                 "l2": "one buffer set reused every step (inputs L2-resident)"},
         "roofline": {
-            "kernel": f"gemm_pair_kernel<{fmt}>" if M > 128 else f"gemm_kernel<{fmt}>",
+            "kernel": f"gemm_pair_kernel<{run_fmt}>" if M > 128 else f"gemm_kernel<{run_fmt}>",
             "bound": "tensor",
             "achieved": round(achieved, 2),
             "peak": round(peak, 1),
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "peak_source": f"{peaks['source']} bf16 sustained {peaks['bf16_sustained']} TFLOP/s x "
-                           f"{NOMINAL_RATIO[fmt]:g} (nominal {fmt}:bf16 dense ratio); the GEMM is "
-                           f"timed by events around its launch inside the timed steps",
-            "peak_burst": round(peak_burst, 1),
-            "frac_of_burst": round(achieved / peak_burst, 4),
+            "peak_kind": "sustained" if sustained else "burst",
+            "peak_source": f"{peaks['source']} bf16 {'sustained' if sustained else 'burst'} "
+                           f"{peaks['bf16_sustained'] if sustained else peaks['bf16']} TFLOP/s x "
+                           f"{NOMINAL_RATIO[run_fmt]:g} (nominal {run_fmt}:bf16 dense ratio); "
+                           f"{'sustained' if sustained else 'burst'} because the GEMM's timed region "
+                           f"was {total_ev_ms:.1f} ms ({'>=' if sustained else '<'} "
+                           f"{SUSTAINED_MIN_MS:.0f} ms); the GEMM is timed by events around its "
+                           f"launch inside the timed steps",
+            "peak_other": round(peak_burst if sustained else peak_sus, 1),
+            "frac_of_other": round(achieved / (peak_burst if sustained else peak_sus), 4),
+            "frac_of_nominal": round(achieved / nominal, 4),
+            "gemm_cycles_per_launch": round(gemm_ms * 1e-3 * gemm_mhz * 1e6) if gemm_mhz else None,
+            "gemm_cycles_note": "in-step GEMM time x median SM clock sampled during that pass",
             "traffic": GEMM_TRAFFIC_BYTES.get(case.name),
             "traffic_unit": "bytes per launch (ncu dram read + write)",
         },
@@ -385,7 +442,7 @@ def run_gpu(args, rank, world, local_rank):
                                        "nominal_peak_tflops": 2250.0,
                                        "measured_burst": round(bf16_tflops / peaks["bf16"], 4)},
         },
-        "clocks": sampler.summary(),
+        "clocks": clocks,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
     }
@@ -559,7 +616,8 @@ def run_stack(args, rank, world, local_rank):
     pass_ms = best_ms / args.steps
     value = whole_job_tflops(world, 1, flops, pass_ms)
     peaks = _peaks()
-    peak = peaks["bf16_sustained"] * NOMINAL_RATIO["nvfp4"]
+    sustained = best_ms >= SUSTAINED_MIN_MS
+    peak = (peaks["bf16_sustained"] if sustained else peaks["bf16"]) * NOMINAL_RATIO["nvfp4"]
     return {
         "metric": METRIC,
         "value": round(value, 2),
@@ -588,7 +646,9 @@ def run_stack(args, rank, world, local_rank):
         "roofline": {"kernel": "whole stack (mixed nvfp4 / bf16 GEMMs)", "bound": "tensor",
                      "achieved": round(value, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
                      "frac": round(value / peak, 4), "traffic": None,
-                     "peak_source": f"{peaks['source']} bf16 sustained x 4 (nvfp4 dense ratio)"},
+                     "peak_kind": "sustained" if sustained else "burst",
+                     "peak_source": f"{peaks['source']} bf16 {'sustained' if sustained else 'burst'} x 4 "
+                                    f"(nvfp4 dense ratio); timed region {best_ms:.0f} ms"},
         "bf16_baseline": {"impl": "torch.addmm bf16 (cuBLAS), the same stack, weights and buffers",
                           "value": round(whole_job_tflops(world, 1, flops, bf16_ms), 2), "unit": UNIT,
                           "ms_per_step": round(bf16_ms, 4),
@@ -663,6 +723,8 @@ def main():
                     help="M,K,N of a seeded random layer instead of a named workload (profiling)")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp8"], help="format for --shape")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--min-dim", type=int, default=None,
+                    help="selective-rule threshold (default 1024; c1 runs with 1, the NVFP4 path)")
     ap.add_argument("--no-tensor-scale", action="store_true",
                     help="NVFP4 without a per-tensor scale (g = 1 for weight and activation)")
     args = ap.parse_args()

@@ -44,6 +44,9 @@ FORMATS = {"nvfp4": NVFP4, "mxfp8": MXFP8, "bf16": BF16}
 # mxq_weight_prepare flags (mxq_weight.flags)
 WEIGHT_KEEP_BF16 = 1
 WEIGHT_NO_TENSOR_SCALE = 2
+WEIGHT_MXFP8_RCEIL = 4
+SCALE_FLOOR = 0
+SCALE_RCEIL = 1
 
 _i64 = ctypes.c_int64
 _ptr = ctypes.c_void_p
@@ -66,9 +69,15 @@ class mxq_weight(ctypes.Structure):
     ]
 
 
+ACT_NONE = 0
+ACT_GELU = 1
+
+
 class mxq_linear_opts(ctypes.Structure):
     _fields_ = [("min_dim", _i64), ("gemm_event_start", ctypes.c_void_p),
-                ("gemm_event_end", ctypes.c_void_p)]
+                ("gemm_event_end", ctypes.c_void_p), ("activation", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("y_amax_dev", ctypes.c_void_p),
+                ("x_amax_dev", ctypes.c_void_p)]
 
 
 def _proto(name, restype, *argtypes):
@@ -87,6 +96,8 @@ _amax = _proto("mxq_amax", _int, _ptr, _i64, _i64, _i64, _ptr, _ptr)
 _quantize_nvfp4 = _proto("mxq_quantize_nvfp4", _int, _ptr, _i64, _i64, _i64, _ptr, _ptr, _ptr,
                          _ptr, _ptr)
 _quantize_mxfp8 = _proto("mxq_quantize_mxfp8", _int, _ptr, _i64, _i64, _i64, _ptr, _ptr, _ptr)
+_quantize_mxfp8_rule = _proto("mxq_quantize_mxfp8_rule", _int, _ptr, _i64, _i64, _i64, _int, _ptr,
+                              _ptr, _ptr)
 _gemm_blockscaled = _proto("mxq_gemm_blockscaled", _int, _int, _i64, _i64, _i64, _ptr, _ptr,
                            _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _i64, _ptr)
 _weight_storage_bytes = _proto("mxq_weight_storage_bytes", _sz, _i64, _i64, _int)
@@ -110,7 +121,7 @@ EXPORTED = [
     "mxq_codes_bytes", "mxq_amax", "mxq_quantize_nvfp4", "mxq_quantize_mxfp8",
     "mxq_gemm_blockscaled", "mxq_weight_storage_bytes", "mxq_weight_prepare",
     "mxq_linear_path", "mxq_linear_workspace_bytes", "mxq_linear", "mxq_get_device_error",
-    "mxq_convert_f32", "mxq_linear_noalloc", "mxq_linear_kernel_count",
+    "mxq_convert_f32", "mxq_linear_noalloc", "mxq_linear_kernel_count", "mxq_quantize_mxfp8_rule",
 ]
 
 #: Capacity of the static device scratch of mxq_linear_noalloc (MXQ_NOALLOC_SCRATCH_BYTES).
@@ -200,10 +211,15 @@ def quantize_nvfp4(x, amax_in, codes, sf, g_out, rows=None, k=None, ld=None, str
                            _addr(g_out), _stream(stream)), "mxq_quantize_nvfp4")
 
 
-def quantize_mxfp8(x, codes, sf, rows=None, k=None, ld=None, stream=None) -> None:
+def quantize_mxfp8(x, codes, sf, rows=None, k=None, ld=None, stream=None, scale_rule=None) -> None:
+    """scale_rule: None / SCALE_FLOOR (the OCP rule) or SCALE_RCEIL."""
     rows, k, ld = _shape2(x, rows, k, ld)
-    _check(_quantize_mxfp8(_addr(x), rows, k, ld, _addr(codes), _addr(sf), _stream(stream)),
-           "mxq_quantize_mxfp8")
+    if scale_rule is None:
+        _check(_quantize_mxfp8(_addr(x), rows, k, ld, _addr(codes), _addr(sf), _stream(stream)),
+               "mxq_quantize_mxfp8")
+    else:
+        _check(_quantize_mxfp8_rule(_addr(x), rows, k, ld, int(scale_rule), _addr(codes), _addr(sf),
+                                    _stream(stream)), "mxq_quantize_mxfp8_rule")
 
 
 def gemm_blockscaled(fmt, M, N, K, a, a_sf, a_g, b, b_sf, b_g, bias, y, ldy=None,
@@ -227,14 +243,19 @@ def weight_prepare(fmt, w, N, K, bias, flags, storage, storage_bytes, stream=Non
     return out
 
 
-def _opts(min_dim, gemm_events=None):
+def _opts(min_dim, gemm_events=None, activation=ACT_NONE, y_amax=None, x_amax=None):
     """mxq_linear_opts; gemm_events: (start, end) torch.cuda.Event pair recorded
-    around the GEMM launch, or None."""
-    if min_dim is None and gemm_events is None:
+    around the GEMM launch, or None; activation / y_amax (device float tensor or
+    address): the producer epilogue; x_amax: the input's known amax."""
+    if (min_dim is None and gemm_events is None and not activation and y_amax is None
+            and x_amax is None):
         return None
     o = mxq_linear_opts(int(min_dim or 0))
     if gemm_events is not None:
         o.gemm_event_start, o.gemm_event_end = (ev.cuda_event for ev in gemm_events)
+    o.activation = int(activation)
+    o.y_amax_dev = _addr(y_amax)
+    o.x_amax_dev = _addr(x_amax)
     return ctypes.byref(o)
 
 
@@ -242,18 +263,20 @@ def linear_path(w: mxq_weight, M: int, min_dim=None) -> int:
     return _linear_path(ctypes.byref(w), M, _opts(min_dim))
 
 
-def linear_kernel_count(w: mxq_weight, M: int, min_dim=None) -> int:
+def linear_kernel_count(w: mxq_weight, M: int, min_dim=None, x_amax=None) -> int:
     """Kernels one mxq_linear call launches for these arguments (-1: no device)."""
-    return _linear_kernel_count(ctypes.byref(w), M, _opts(min_dim))
+    return _linear_kernel_count(ctypes.byref(w), M, _opts(min_dim, x_amax=x_amax))
 
 
 def linear_workspace_bytes(M: int, K: int, fmt) -> int:
     return _linear_workspace_bytes(M, K, _fmt(fmt))
 
 
-def linear(w: mxq_weight, x, M, y, ws, ws_bytes, min_dim=None, stream=None, gemm_events=None) -> None:
+def linear(w: mxq_weight, x, M, y, ws, ws_bytes, min_dim=None, stream=None, gemm_events=None,
+           activation=ACT_NONE, y_amax=None, x_amax=None) -> None:
     _check(_linear(ctypes.byref(w), _addr(x), M, _addr(y), _addr(ws), ws_bytes,
-                   _opts(min_dim, gemm_events), _stream(stream)), "mxq_linear")
+                   _opts(min_dim, gemm_events, activation, y_amax, x_amax), _stream(stream)),
+           "mxq_linear")
 
 
 def linear_noalloc(w: mxq_weight, x, M, y, min_dim=None, stream=None) -> None:
@@ -279,13 +302,16 @@ class Weight:
     into (kept alive here).  Allocation is torch's; quantisation runs in
     mxq_weight_prepare."""
 
-    def __init__(self, w, bias=None, fmt="nvfp4", keep_bf16=False, tensor_scale=True, stream=None):
+    def __init__(self, w, bias=None, fmt="nvfp4", keep_bf16=False, tensor_scale=True,
+                 mxfp8_rceil=False, stream=None):
         """tensor_scale=False: NVFP4 without a per-tensor scale (g = 1 for the
-        weight and every activation)."""
+        weight and every activation); mxfp8_rceil=True: MXFP8 with the ceiling
+        scale rule."""
         import torch
         N, K = w.shape
         self.w, self.bias, self.fmt = w, bias, _fmt(fmt)
-        flags = (WEIGHT_KEEP_BF16 if keep_bf16 else 0) | (0 if tensor_scale else WEIGHT_NO_TENSOR_SCALE)
+        flags = ((WEIGHT_KEEP_BF16 if keep_bf16 else 0) | (0 if tensor_scale else WEIGHT_NO_TENSOR_SCALE)
+                 | (WEIGHT_MXFP8_RCEIL if mxfp8_rceil else 0))
         nbytes = weight_storage_bytes(N, K, self.fmt) if not keep_bf16 else 0
         self.storage = (torch.empty(max(nbytes, 256), dtype=torch.uint8, device=w.device)
                         if nbytes else None)

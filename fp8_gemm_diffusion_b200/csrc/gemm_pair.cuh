@@ -135,9 +135,20 @@ struct PairArgs {
   const float* a_g;
   const float* b_g;
   const __nv_bfloat16* bias;
+  int act;                // EPI != 0 only: 1 = GELU on alpha * acc + bias before the bf16 rounding
+  unsigned int* y_amax;   // EPI != 0 only: max |y| over the bf16 outputs, folded in with atomicMax
 };
 
-template <Fmt F, int BN>
+// GELU with the exact error function, x * Phi(x), in fp32.
+__device__ __forceinline__ float gelu_erf(float x) {
+  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+}
+
+// EPI = 0: the plain epilogue.  EPI = 1: the producer epilogue of a layer
+// whose output feeds the next layer's quantiser: optional GELU, and the
+// output's max |y| folded into one device word, so that the next layer's
+// NVFP4 quantisation needs no amax pass over its input.
+template <Fmt F, int BN, int EPI = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b,
@@ -428,6 +439,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
     float alpha = 1.0f;
     if constexpr (F == Fmt::NVFP4) alpha = (*args.a_g) * (*args.b_g);
     const bool bias_vec = args.bias != nullptr && (reinterpret_cast<uintptr_t>(args.bias) & 15u) == 0;
+    float ymax = 0.0f;  // EPI != 0: max |y| of this thread's outputs
     for (int i_tile = 0; i_tile < my_tiles; ++i_tile) {
       const int tile = pair + i_tile * num_pairs;
       int mt, nt;
@@ -486,7 +498,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
             if constexpr (F == Fmt::NVFP4) { v0 *= alpha; v1 *= alpha; }
             v0 += __uint_as_float(bw[e] << 16);
             v1 += __uint_as_float(bw[e] & 0xFFFF0000u);
+            if constexpr (EPI != 0) {
+              if (args.act == 1) {
+                v0 = gelu_erf(v0);
+                v1 = gelu_erf(v1);
+              }
+            }
             const __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
+            if constexpr (EPI != 0) {
+              // rows and columns past the edge hold no output: leave them out
+              const int cc = col_w + c;
+              if (row0 + lane < M && cc < N) ymax = fmaxf(ymax, fabsf(__low2float(hv)));
+              if (row0 + lane < M && cc + 1 < N) ymax = fmaxf(ymax, fabsf(__high2float(hv)));
+            }
             pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
           }
           static_assert(C::EPI_SUB == 32, "staging swizzle");
@@ -503,6 +527,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
           bulk_commit_group();
         }
       }
+    }
+    if constexpr (EPI != 0) {
+      // non-negative floats order like their bit patterns
+      const unsigned int m = __reduce_max_sync(0xffffffffu, __float_as_uint(ymax));
+      if (lane == 0 && args.y_amax != nullptr) atomicMax(args.y_amax, m);
     }
     if (lane == 0) bulk_wait_all();
   }

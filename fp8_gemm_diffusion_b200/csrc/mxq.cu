@@ -252,12 +252,18 @@ mxq_status launch_quant_nvfp4_fused(const void* x, int64_t rows, int64_t k, int6
 }
 
 mxq_status launch_quant_mxfp8(const void* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
-                              uint8_t* sf, cudaStream_t s, int sms) {
+                              uint8_t* sf, cudaStream_t s, int sms, int rceil = 0) {
   cudaError_t e = launch_pdl(mxq::quantize_mxfp8_kernel, dim3(quant_grid(rows, sms)),
                              dim3(mxq::kQuantThreads), 0, s, static_cast<const __nv_bfloat16*>(x),
-                             static_cast<int>(rows), static_cast<int>(k), ld, codes, sf);
+                             static_cast<int>(rows), static_cast<int>(k), ld, codes, sf, rceil);
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
+
+// Epilogue options of the pair kernel's producer variant (mxq_linear_opts).
+struct Epilogue {
+  int act = 0;             // MXQ_ACT_*
+  float* y_amax = nullptr; // receives max |y| (atomicMax on the bits; zeroed by the caller)
+};
 
 template <mxq::Fmt F, int BN>
 mxq_status launch_gemm_bn(int dev, int sms, int slot, int64_t M, int64_t N, int64_t K,
@@ -308,13 +314,13 @@ mxq_status launch_gemm_bn(int dev, int sms, int slot, int64_t M, int64_t N, int6
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
-template <mxq::Fmt F, int BN>
+template <mxq::Fmt F, int BN, int EPI>
 mxq_status launch_gemm_pair(int dev, int sms, int slot, int64_t M, int64_t N, int64_t K,
                             const void* a, const uint8_t* a_sf, const float* a_g, const void* b,
                             const uint8_t* b_sf, const float* b_g, const void* bias, void* y,
-                            int64_t ldy, cudaStream_t s) {
+                            int64_t ldy, const Epilogue& ep, cudaStream_t s) {
   using C = mxq::PairCfg<F, BN>;
-  auto kern = mxq::gemm_pair_kernel<F, BN>;
+  auto kern = mxq::gemm_pair_kernel<F, BN, EPI>;
   const uint32_t bit = 1u << slot;
   if (!(g_dev[dev].smem_attr_set.load(std::memory_order_acquire) & bit)) {
     cudaError_t e =
@@ -359,6 +365,8 @@ mxq_status launch_gemm_pair(int dev, int sms, int slot, int64_t M, int64_t N, in
   args.a_g = a_g;
   args.b_g = b_g;
   args.bias = static_cast<const __nv_bfloat16*>(bias);
+  args.act = ep.act;
+  args.y_amax = reinterpret_cast<unsigned int*>(ep.y_amax);
   const int64_t tiles = ((M + C::BM - 1) / C::BM) * ((N + BN - 1) / BN);
   const int64_t pairs = sms / 2;
   const int grid = 2 * static_cast<int>(tiles < pairs ? tiles : pairs);
@@ -367,34 +375,48 @@ mxq_status launch_gemm_pair(int dev, int sms, int slot, int64_t M, int64_t N, in
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
+template <int EPI>
+mxq_status launch_gemm_pairs(mxq_format f, int dev, int sms, int64_t M, int64_t N, int64_t K,
+                             const void* a, const uint8_t* a_sf, const float* a_g, const void* b,
+                             const uint8_t* b_sf, const float* b_g, const void* bias, void* y,
+                             int64_t ldy, const Epilogue& ep, cudaStream_t s) {
+  // slots 6-11: plain epilogue; 12-17: producer epilogue
+  const int base = EPI ? 12 : 6;
+  switch (f) {
+    case MXQ_NVFP4:
+      if (N > 128)
+        return launch_gemm_pair<mxq::Fmt::NVFP4, 256, EPI>(dev, sms, base, M, N, K, a, a_sf, a_g, b,
+                                                           b_sf, b_g, bias, y, ldy, ep, s);
+      return launch_gemm_pair<mxq::Fmt::NVFP4, 128, EPI>(dev, sms, base + 1, M, N, K, a, a_sf, a_g, b,
+                                                         b_sf, b_g, bias, y, ldy, ep, s);
+    case MXQ_MXFP8:
+      if (N > 128)
+        return launch_gemm_pair<mxq::Fmt::MXFP8, 256, EPI>(dev, sms, base + 2, M, N, K, a, a_sf, a_g, b,
+                                                           b_sf, b_g, bias, y, ldy, ep, s);
+      return launch_gemm_pair<mxq::Fmt::MXFP8, 128, EPI>(dev, sms, base + 3, M, N, K, a, a_sf, a_g, b,
+                                                         b_sf, b_g, bias, y, ldy, ep, s);
+    case MXQ_BF16:
+      if (N > 128)
+        return launch_gemm_pair<mxq::Fmt::BF16, 256, EPI>(dev, sms, base + 4, M, N, K, a, a_sf, a_g, b,
+                                                          b_sf, b_g, bias, y, ldy, ep, s);
+      return launch_gemm_pair<mxq::Fmt::BF16, 128, EPI>(dev, sms, base + 5, M, N, K, a, a_sf, a_g, b,
+                                                        b_sf, b_g, bias, y, ldy, ep, s);
+  }
+  return MXQ_ERR_INVALID_ARG;
+}
+
 mxq_status launch_gemm(mxq_format f, int dev, int sms, int64_t M, int64_t N, int64_t K,
                        const void* a, const uint8_t* a_sf, const float* a_g, const void* b,
                        const uint8_t* b_sf, const float* b_g, const void* bias, void* y,
-                       int64_t ldy, cudaStream_t s) {
+                       int64_t ldy, cudaStream_t s, const Epilogue& ep = Epilogue{}) {
+  const bool producer = ep.act != 0 || ep.y_amax != nullptr;
   if (M > 128) {
     // CTA-pair kernel (M = 256 MMAs)
-    switch (f) {
-      case MXQ_NVFP4:
-        if (N > 128)
-          return launch_gemm_pair<mxq::Fmt::NVFP4, 256>(dev, sms, 6, M, N, K, a, a_sf, a_g, b, b_sf,
-                                                        b_g, bias, y, ldy, s);
-        return launch_gemm_pair<mxq::Fmt::NVFP4, 128>(dev, sms, 7, M, N, K, a, a_sf, a_g, b, b_sf,
-                                                      b_g, bias, y, ldy, s);
-      case MXQ_MXFP8:
-        if (N > 128)
-          return launch_gemm_pair<mxq::Fmt::MXFP8, 256>(dev, sms, 8, M, N, K, a, a_sf, a_g, b, b_sf,
-                                                        b_g, bias, y, ldy, s);
-        return launch_gemm_pair<mxq::Fmt::MXFP8, 128>(dev, sms, 9, M, N, K, a, a_sf, a_g, b, b_sf,
-                                                      b_g, bias, y, ldy, s);
-      case MXQ_BF16:
-        if (N > 128)
-          return launch_gemm_pair<mxq::Fmt::BF16, 256>(dev, sms, 10, M, N, K, a, a_sf, a_g, b, b_sf,
-                                                       b_g, bias, y, ldy, s);
-        return launch_gemm_pair<mxq::Fmt::BF16, 128>(dev, sms, 11, M, N, K, a, a_sf, a_g, b, b_sf,
-                                                     b_g, bias, y, ldy, s);
-    }
-    return MXQ_ERR_INVALID_ARG;
+    if (producer)
+      return launch_gemm_pairs<1>(f, dev, sms, M, N, K, a, a_sf, a_g, b, b_sf, b_g, bias, y, ldy, ep, s);
+    return launch_gemm_pairs<0>(f, dev, sms, M, N, K, a, a_sf, a_g, b, b_sf, b_g, bias, y, ldy, ep, s);
   }
+  if (producer) return MXQ_ERR_UNSUPPORTED_SHAPE;  // the single-CTA kernel has the plain epilogue only
   switch (f) {
     case MXQ_NVFP4:
       if (N % 192 == 0)
@@ -513,6 +535,13 @@ mxq_status mxq_quantize_nvfp4(const void* x_bf16, int64_t rows, int64_t k, int64
 
 mxq_status mxq_quantize_mxfp8(const void* x_bf16, int64_t rows, int64_t k, int64_t ld,
                               uint8_t* codes, uint8_t* sf_swz, mxq_stream_t stream) {
+  return mxq_quantize_mxfp8_rule(x_bf16, rows, k, ld, MXQ_SCALE_FLOOR, codes, sf_swz, stream);
+}
+
+mxq_status mxq_quantize_mxfp8_rule(const void* x_bf16, int64_t rows, int64_t k, int64_t ld,
+                                   int scale_rule, uint8_t* codes, uint8_t* sf_swz,
+                                   mxq_stream_t stream) {
+  if (scale_rule != MXQ_SCALE_FLOOR && scale_rule != MXQ_SCALE_RCEIL) return MXQ_ERR_INVALID_ARG;
   mxq_status st = check_bf16_matrix(x_bf16, rows, k, ld);
   if (st != MXQ_OK) return st;
   if (rows > 0 && k > 0 && (codes == nullptr || sf_swz == nullptr)) return MXQ_ERR_INVALID_ARG;
@@ -522,14 +551,19 @@ mxq_status mxq_quantize_mxfp8(const void* x_bf16, int64_t rows, int64_t k, int64
   if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
   if (rows == 0 || k == 0) return MXQ_OK;
   return launch_quant_mxfp8(x_bf16, rows, k, ld, codes, sf_swz,
-                            reinterpret_cast<cudaStream_t>(stream), sms);
+                            reinterpret_cast<cudaStream_t>(stream), sms,
+                            scale_rule == MXQ_SCALE_RCEIL ? 1 : 0);
 }
 
-mxq_status mxq_gemm_blockscaled(mxq_format f, int64_t M, int64_t N, int64_t K,
-                                const void* a_codes, const uint8_t* a_sf, const float* a_g_dev,
-                                const void* b_codes, const uint8_t* b_sf, const float* b_g_dev,
-                                const void* bias_bf16, void* y_bf16, int64_t ldy,
-                                mxq_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// mxq_gemm_blockscaled with an epilogue (the producer variant for mxq_linear).
+mxq_status gemm_checked(mxq_format f, int64_t M, int64_t N, int64_t K, const void* a_codes,
+                        const uint8_t* a_sf, const float* a_g_dev, const void* b_codes,
+                        const uint8_t* b_sf, const float* b_g_dev, const void* bias_bf16,
+                        void* y_bf16, int64_t ldy, mxq_stream_t stream, const Epilogue& ep) {
   if (!valid_format(f)) return MXQ_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0) return MXQ_ERR_INVALID_ARG;
   if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return MXQ_ERR_UNSUPPORTED_SHAPE;
@@ -554,7 +588,20 @@ mxq_status mxq_gemm_blockscaled(mxq_format f, int64_t M, int64_t N, int64_t K,
   if (!nonempty) return MXQ_OK;
   if ((st = get_encoder()) != MXQ_OK) return st;
   return launch_gemm(f, dev, sms, M, N, K, a_codes, a_sf, a_g_dev, b_codes, b_sf, b_g_dev,
-                     bias_bf16, y_bf16, ldy, reinterpret_cast<cudaStream_t>(stream));
+                     bias_bf16, y_bf16, ldy, reinterpret_cast<cudaStream_t>(stream), ep);
+}
+
+}  // namespace
+
+extern "C" {
+
+mxq_status mxq_gemm_blockscaled(mxq_format f, int64_t M, int64_t N, int64_t K,
+                                const void* a_codes, const uint8_t* a_sf, const float* a_g_dev,
+                                const void* b_codes, const uint8_t* b_sf, const float* b_g_dev,
+                                const void* bias_bf16, void* y_bf16, int64_t ldy,
+                                mxq_stream_t stream) {
+  return gemm_checked(f, M, N, K, a_codes, a_sf, a_g_dev, b_codes, b_sf, b_g_dev, bias_bf16, y_bf16,
+                      ldy, stream, Epilogue{});
 }
 
 size_t mxq_weight_storage_bytes(int64_t N, int64_t K, mxq_format f) {
@@ -567,10 +614,13 @@ mxq_status mxq_weight_prepare(mxq_format f, const void* w_bf16, int64_t N, int64
                               const void* bias_bf16, int flags, void* storage,
                               size_t storage_bytes, mxq_weight* out, mxq_stream_t stream) {
   if (out == nullptr || !valid_format(f)) return MXQ_ERR_INVALID_ARG;
-  if (flags & ~(MXQ_WEIGHT_KEEP_BF16 | MXQ_WEIGHT_NO_TENSOR_SCALE)) return MXQ_ERR_INVALID_ARG;
+  if (flags & ~(MXQ_WEIGHT_KEEP_BF16 | MXQ_WEIGHT_NO_TENSOR_SCALE | MXQ_WEIGHT_MXFP8_RCEIL))
+    return MXQ_ERR_INVALID_ARG;
   const bool keep_bf16 = (flags & MXQ_WEIGHT_KEEP_BF16) != 0;
   const bool no_tensor_scale = (flags & MXQ_WEIGHT_NO_TENSOR_SCALE) != 0;
+  const int rceil = (flags & MXQ_WEIGHT_MXFP8_RCEIL) ? 1 : 0;
   if (no_tensor_scale && f != MXQ_NVFP4) return MXQ_ERR_INVALID_ARG;
+  if (rceil && f != MXQ_MXFP8) return MXQ_ERR_INVALID_ARG;
   mxq_status st = check_bf16_matrix(w_bf16, N, K, K);
   if (st != MXQ_OK) return st;
   if (bias_bf16 != nullptr && (reinterpret_cast<uintptr_t>(bias_bf16) & 1u)) return MXQ_ERR_ALIGNMENT;
@@ -614,7 +664,7 @@ mxq_status mxq_weight_prepare(mxq_format f, const void* w_bf16, int64_t N, int64
       w.g_dev = g;
       w.amax_dev = amax;
     } else {
-      if (N > 0 && K > 0 && (st = launch_quant_mxfp8(w_bf16, N, K, K, codes, sf, s, sms)) != MXQ_OK)
+      if (N > 0 && K > 0 && (st = launch_quant_mxfp8(w_bf16, N, K, K, codes, sf, s, sms, rceil)) != MXQ_OK)
         return st;
     }
     w.codes = codes;
@@ -652,18 +702,43 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
   const int path = mxq_linear_path(w, M, opts);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  Epilogue ep;
+  const float* x_amax = nullptr;
   if (opts != nullptr) {
     if ((opts->gemm_event_start == nullptr) != (opts->gemm_event_end == nullptr))
       return MXQ_ERR_INVALID_ARG;
     ev0 = static_cast<cudaEvent_t>(opts->gemm_event_start);
     ev1 = static_cast<cudaEvent_t>(opts->gemm_event_end);
+    if (opts->activation != MXQ_ACT_NONE && opts->activation != MXQ_ACT_GELU) return MXQ_ERR_INVALID_ARG;
+    ep.act = opts->activation;
+    ep.y_amax = opts->y_amax_dev;
+    x_amax = opts->x_amax_dev;
+    if ((reinterpret_cast<uintptr_t>(ep.y_amax) & 3u) || (reinterpret_cast<uintptr_t>(x_amax) & 3u))
+      return MXQ_ERR_ALIGNMENT;
+    if (ep.y_amax != nullptr && static_cast<const float*>(ep.y_amax) == x_amax) return MXQ_ERR_INVALID_ARG;
   }
+  const bool producer = ep.act != MXQ_ACT_NONE || ep.y_amax != nullptr;
+  // the producer epilogue lives in the CTA-pair kernel (M > 128) only
+  if (producer && M > 0 && M <= 128 && N > 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  // max |y| is folded in with atomicMax: it starts from 0 (also the value for
+  // an empty y), set on the stream once every check has passed
+  auto zero_y_amax = [&]() -> mxq_status {
+    if (ep.y_amax == nullptr) return MXQ_OK;
+    const cudaError_t e = cudaMemsetAsync(ep.y_amax, 0, sizeof(float), s);
+    return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
+  };
   if (path == MXQ_BF16) {
     if (M > 0 && N > 0 && w->w_bf16 == nullptr) return MXQ_ERR_INVALID_ARG;
+    if (!aligned16(w->w_bf16)) return MXQ_ERR_ALIGNMENT;
+    if (w->bias_bf16 != nullptr && (reinterpret_cast<uintptr_t>(w->bias_bf16) & 1u)) return MXQ_ERR_ALIGNMENT;
+    if (K == 0) return MXQ_ERR_UNSUPPORTED_SHAPE;  // as mxq_gemm_blockscaled
+    int dev, sms;
+    if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+    if ((st = zero_y_amax()) != MXQ_OK) return st;
     cudaError_t e;
     if (ev0 != nullptr && (e = cudaEventRecord(ev0, s)) != cudaSuccess) return cuda_fail(e);
-    st = mxq_gemm_blockscaled(MXQ_BF16, M, N, K, x_bf16, nullptr, nullptr, w->w_bf16, nullptr,
-                              nullptr, w->bias_bf16, y_bf16, N, stream);
+    st = gemm_checked(MXQ_BF16, M, N, K, x_bf16, nullptr, nullptr, w->w_bf16, nullptr, nullptr,
+                      w->bias_bf16, y_bf16, N, stream, ep);
     if (st == MXQ_OK && ev1 != nullptr && (e = cudaEventRecord(ev1, s)) != cudaSuccess)
       return cuda_fail(e);
     return st;
@@ -677,6 +752,7 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
   if (ws_bytes < l.total) return MXQ_ERR_WORKSPACE;
   int dev, sms;
   if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+  if ((st = zero_y_amax()) != MXQ_OK) return st;
   if (M == 0 || N == 0) return MXQ_OK;
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* amax = reinterpret_cast<float*>(base);
@@ -686,6 +762,10 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
   if (f == MXQ_NVFP4 && (w->flags & MXQ_WEIGHT_NO_TENSOR_SCALE)) {
     // no per-tensor scale: one pass, g = 1 (no amax values to reduce)
     if ((st = launch_quant_nvfp4(x_bf16, M, K, K, nullptr, 0, codes, sf, g, amax, s, sms)) != MXQ_OK)
+      return st;
+  } else if (f == MXQ_NVFP4 && x_amax != nullptr) {
+    // the input's amax is known (e.g. from the producing layer's epilogue): one pass
+    if ((st = launch_quant_nvfp4(x_bf16, M, K, K, x_amax, 1, codes, sf, g, amax, s, sms)) != MXQ_OK)
       return st;
   } else if (f == MXQ_NVFP4) {
     float* partials = reinterpret_cast<float*>(base + kPartialsOff);
@@ -705,13 +785,14 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
         return st;
     }
   } else {
-    if ((st = launch_quant_mxfp8(x_bf16, M, K, K, codes, sf, s, sms)) != MXQ_OK) return st;
+    const int rceil = (w->flags & MXQ_WEIGHT_MXFP8_RCEIL) ? 1 : 0;
+    if ((st = launch_quant_mxfp8(x_bf16, M, K, K, codes, sf, s, sms, rceil)) != MXQ_OK) return st;
   }
   if ((st = get_encoder()) != MXQ_OK) return st;
   cudaError_t e;
   if (ev0 != nullptr && (e = cudaEventRecord(ev0, s)) != cudaSuccess) return cuda_fail(e);
   st = launch_gemm(f, dev, sms, M, N, K, codes, sf, g, w->codes, w->sf, w->g_dev, w->bias_bf16,
-                   y_bf16, N, s);
+                   y_bf16, N, s, ep);
   if (st == MXQ_OK && ev1 != nullptr && (e = cudaEventRecord(ev1, s)) != cudaSuccess)
     return cuda_fail(e);
   return st;
@@ -722,6 +803,7 @@ int mxq_linear_kernel_count(const mxq_weight* w, int64_t M, const mxq_linear_opt
   const int path = mxq_linear_path(w, M, opts);
   if (path == MXQ_BF16) return 1;
   if (path == MXQ_MXFP8 || (w->flags & MXQ_WEIGHT_NO_TENSOR_SCALE)) return 2;
+  if (opts != nullptr && opts->x_amax_dev != nullptr) return 2;
   int dev, sms;
   if (current_device(&dev, &sms) != MXQ_OK) return -1;
   return plan_fused(M, w->K, sms).grid > 0 ? 2 : 3;

@@ -495,7 +495,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 // -------------------------------------------------------------- MXFP8
 __global__ void __launch_bounds__(kQuantThreads)
     quantize_mxfp8_kernel(const __nv_bfloat16* __restrict__ x, int rows, int k, int64_t ld,
-                          uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+                          uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, int rceil) {
   grid_dep_wait();
   grid_dep_launch();
   const int lane = threadIdx.x & 31;
@@ -522,7 +522,13 @@ __global__ void __launch_bounds__(kQuantThreads)
         bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
         bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));  // 32-element block
         int X = -127;
-        if (bmax > 0.0f) X = min(max(floor_log2_f32(bmax) - 8, -127), 127);
+        if (bmax > 0.0f) {
+          int e = floor_log2_f32(bmax) - 8;
+          // ceiling rule: the smallest X with bmax <= 448 * 2^X, i.e. one more
+          // when bmax > 1.75 * 2^(e + 8) (exact in double)
+          if (rceil && static_cast<double>(bmax) > ldexp(1.75, e + 8)) e += 1;
+          X = min(max(e, -127), 127);
+        }
         const float mult = exp2_int(-X);
         uint2 out;
         out.x = cvt_e4m3x2(f[0] * mult, f[1] * mult) | (cvt_e4m3x2(f[2] * mult, f[3] * mult) << 16);

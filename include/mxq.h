@@ -133,6 +133,17 @@ mxq_status mxq_quantize_nvfp4(const void* x_bf16, int64_t rows, int64_t k, int64
 mxq_status mxq_quantize_mxfp8(const void* x_bf16, int64_t rows, int64_t k, int64_t ld,
                               uint8_t* codes, uint8_t* sf_swz, mxq_stream_t stream);
 
+/* MXFP8 scale rules: the OCP floor rule above, or the ceiling rule (TorchAO's
+ * RCEIL; not in the pages): X = the smallest integer with bamax <= 448 * 2^X,
+ * clamped to [-127, 127], so no element saturates. */
+enum { MXQ_SCALE_FLOOR = 0, MXQ_SCALE_RCEIL = 1 };
+
+/* mxq_quantize_mxfp8 with a scale rule (MXQ_SCALE_*; other values ->
+ * INVALID_ARG).  Same arguments, outputs and errors otherwise. */
+mxq_status mxq_quantize_mxfp8_rule(const void* x_bf16, int64_t rows, int64_t k, int64_t ld,
+                                   int scale_rule, uint8_t* codes, uint8_t* sf_swz,
+                                   mxq_stream_t stream);
+
 /* ------------------------------------------------------------- GEMM ----- */
 
 /*
@@ -162,8 +173,10 @@ mxq_status mxq_gemm_blockscaled(mxq_format f, int64_t M, int64_t N, int64_t K,
 /* Flags of mxq_weight_prepare and mxq_weight.flags. */
 enum {
   MXQ_WEIGHT_KEEP_BF16 = 1,       /* always run this layer as a bf16 GEMM          */
-  MXQ_WEIGHT_NO_TENSOR_SCALE = 2  /* NVFP4 without a per-tensor scale: g = 1 for
+  MXQ_WEIGHT_NO_TENSOR_SCALE = 2, /* NVFP4 without a per-tensor scale: g = 1 for
                                      both W and every activation (no amax pass)    */
+  MXQ_WEIGHT_MXFP8_RCEIL = 4      /* MXFP8 with the ceiling scale rule for W and
+                                     every activation                              */
 };
 
 /*
@@ -197,12 +210,18 @@ size_t mxq_weight_storage_bytes(int64_t N, int64_t K, mxq_format f);
  * quantised (storage may be NULL) and the layer always runs in bf16.  With
  * MXQ_WEIGHT_NO_TENSOR_SCALE (NVFP4 only, else INVALID_ARG) W is quantised
  * with g_W = 1 and mxq_linear quantises activations with g = 1 (no amax).
+ * With MXQ_WEIGHT_MXFP8_RCEIL (MXFP8 only, else INVALID_ARG) W and every
+ * activation of the layer use the ceiling scale rule (MXQ_SCALE_RCEIL).
  */
 mxq_status mxq_weight_prepare(mxq_format f, const void* w_bf16, int64_t N, int64_t K,
                               const void* bias_bf16, int flags, void* storage,
                               size_t storage_bytes, mxq_weight* out, mxq_stream_t stream);
 
-/* Options of mxq_linear.  A NULL pointer means the defaults. */
+/* Activation applied in the GEMM epilogue (mxq_linear_opts.activation). */
+enum { MXQ_ACT_NONE = 0, MXQ_ACT_GELU = 1 /* x * Phi(x), exact erf */ };
+
+/* Options of mxq_linear.  A NULL pointer means the defaults; a zeroed struct
+ * is the defaults too. */
 typedef struct mxq_linear_opts {
   int64_t min_dim;          /* bf16 when min(M,K,N) < min_dim; 0 -> 1024 (the article's rule) */
   void* gemm_event_start;   /* optional cudaEvent_t (NULL: none): mxq_linear records it on the
@@ -210,6 +229,18 @@ typedef struct mxq_linear_opts {
                                after, so a caller can time the GEMM inside a step.  Both or
                                neither; the events stay the caller's. */
   void* gemm_event_end;
+  /* Producer epilogue (kernel fusion of the activation and of the next layer's amax; the
+   * devin.kr Blackwell FLUX page, section "연산 효율화와 가속 기술": activation functions fused
+   * into the custom GEMM).  Available on the CTA-pair GEMM (M > 128); with M <= 128 either
+   * option gives MXQ_ERR_UNSUPPORTED_SHAPE. */
+  int32_t activation;       /* MXQ_ACT_*: applied to alpha*acc + bias before the bf16 rounding */
+  int32_t reserved;         /* 0 */
+  float* y_amax_dev;        /* optional device float (4-byte aligned): receives max |y| over the
+                               bf16 output (zeroed on the stream first) */
+  /* Consumer side: the input's amax already known (e.g. the producing layer's y_amax_dev).
+   * The NVFP4 path (with a per-tensor scale) then skips its amax pass: one quantisation
+   * kernel reads x once.  Ignored by the other paths.  Must not alias y_amax_dev. */
+  const float* x_amax_dev;
 } mxq_linear_opts;
 
 /*

@@ -14,15 +14,13 @@ Plain numpy, written to be checked by eye against the definitions:
 * ``gemm``     - float64 reference of the quantised linear and its tolerance.
 * ``dispatch`` - the selective-quantisation rule.
 * ``producer`` - a linear layer with the GELU activation fused into its
-  epilogue, and that epilogue's error scale (the oracle of the fused-producer
-  kernel that comes next; no GPU kernel uses it yet).
+  epilogue, and that epilogue's error scale.
 
 Every function is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle_*.py`` to facts other than itself (code tables, tie cases,
 exact blocks, closed forms, brute force on tiny shapes, an independent library
-cast).  The scale-factor byte layout is the one part with no such pin: it is
-checked only indirectly, through GEMM parity on the GPU (parity unpinned on
-the CPU side).
+cast, byte offsets of the scale-factor layout worked by hand from its
+published description).
 """
 
 from . import formats, quant, gemm, dispatch, producer  # noqa: F401

@@ -243,3 +243,40 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert got[(st, "size")] == ctypes.sizeof(cls), st
         for n in fields[st]:
             assert got[(st, n)] == getattr(cls, n).offset, (st, n)
+
+
+def test_producer_and_known_amax_options_are_checked_on_the_host():
+    N = K = M = 1024
+    need = mxq.linear_workspace_bytes(M, K, "nvfp4")
+    w = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=N, K=K, w_bf16=dev(N * K * 2), bias_bf16=None,
+                       codes=dev(N * K // 2), sf=dev(mxq.sf_bytes(N, K, "nvfp4")), g_dev=dev(4),
+                       amax_dev=dev(4))
+    x, y, ws, f4 = dev(M * K * 2), dev(M * N * 2), dev(need), dev(16)
+
+    def call(M_=M, **kw):
+        return mxq._linear(mxq.ctypes.byref(w), x, M_, y, ws, need, mxq._opts(None, **kw), mxq._stream(None))
+
+    assert call(activation=7) == mxq.ERR_INVALID_ARG
+    assert call(y_amax=f4 + 2) == mxq.ERR_ALIGNMENT
+    assert call(x_amax=f4 + 1) == mxq.ERR_ALIGNMENT
+    assert call(y_amax=f4, x_amax=f4) == mxq.ERR_INVALID_ARG            # must not alias
+    assert call(M_=128, activation=mxq.ACT_GELU) == mxq.ERR_UNSUPPORTED_SHAPE   # single-CTA GEMM
+    assert call(M_=64, y_amax=f4) == mxq.ERR_UNSUPPORTED_SHAPE
+    # a known amax removes the amax pass: quantiser + GEMM
+    assert mxq.linear_kernel_count(w, 4096, x_amax=f4) == 2
+    if not torch.cuda.is_available():
+        assert call(activation=mxq.ACT_GELU, y_amax=f4) == mxq.ERR_ARCH  # past every argument check
+
+
+def test_rceil_flag_and_scale_rule_checks():
+    out = mxq.mxq_weight()
+    w16 = dev(1024 * 1024 * 2)
+    for fmt in (mxq.NVFP4, mxq.BF16):
+        st = mxq._weight_prepare(fmt, w16, 1024, 1024, None, mxq.WEIGHT_MXFP8_RCEIL, None, 0,
+                                 mxq.ctypes.byref(out), None)
+        assert st == mxq.ERR_INVALID_ARG, fmt
+    assert _st(mxq.quantize_mxfp8, dev(SMALL), dev(SMALL), dev(SMALL), 4, 128, 128, None, 2) \
+        == mxq.ERR_INVALID_ARG
+    if not torch.cuda.is_available():
+        assert _st(mxq.quantize_mxfp8, dev(SMALL), dev(SMALL), dev(SMALL), 4, 128, 128, None,
+                   mxq.SCALE_RCEIL) == mxq.ERR_ARCH

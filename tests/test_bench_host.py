@@ -40,15 +40,30 @@ def test_reference_arm_for_the_stack_is_unavailable():
     assert d["impl"] == "reference" and "unavailable" in d
 
 
-def test_clock_summary_flags_throttling():
+def test_clock_summary_flags_throttling_and_counts_windows():
     s = bench.ClockSampler.__new__(bench.ClockSampler)
-    s._h, s.max_mhz = object(), 1965
-    s.samples = [1800, 1900, 1965]
-    s.reasons = 0x4 | 0x1  # sw_power_cap, and gpu_idle which is not reported
-    out = s.summary()
-    assert out == {"sm_mhz": 1900.0, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"], "samples": 3}
+    s._h, s.max_mhz, s.period = object(), 1965, 0.0002
+    # (host time, SM MHz, reason bits): sw_power_cap once, gpu_idle (not reported) once
+    s.samples = [(0.0, 1800, 0x1), (1.0, 1900, 0x4), (2.0, 1965, 0), (3.0, 1500, 0)]
+    s.windows = {}
+    s.mark("headline", 0.5, 2.5)
+    s.mark("other", 2.5, 3.5)
+    out = s.summary("headline")
+    assert out["sm_mhz"] == 1850.0 and out["samples"] == 4 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap"]
+    assert out["windows"]["headline"] == {"sm_mhz": 1932.5, "reasons": ["sw_power_cap"], "samples": 2,
+                                          "sm_mhz_min": 1900}
+    assert out["windows"]["other"]["samples"] == 1 and out["windows"]["other"]["reasons"] == []
+    assert out["sm_mhz_headline"] == 1932.5 and out["samples_headline"] == 2
     s._h = None
     assert s.summary()["reasons"] == ["unavailable"]
+
+
+def test_sustained_peak_needs_a_long_timed_region():
+    # the denominator switches to the sustained figure only for a GEMM timed
+    # inside a region of at least a second
+    assert bench.SUSTAINED_MIN_MS >= 1000.0
+    assert bench.NOMINAL_RATIO == {"nvfp4": 4.0, "mxfp8": 2.0, "bf16": 1.0}
 
 
 def test_peaks_come_from_the_measured_file_or_the_fallback():
