@@ -63,10 +63,7 @@ NOMINAL_RATIO = {"nvfp4": 4.0, "mxfp8": 2.0, "bf16": 1.0}
 # DRAM bytes (read + write) of one launch of the roofline's kernel, from one
 # ncu capture of the committed kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum); None where no capture of the current kernel exists.
-GEMM_TRAFFIC_BYTES = {
-    "c3_nvfp4_4608x3072x12288": 29_289_728 + 63_094_784,  # gemm_pair_kernel<NVFP4, 256>
-    "c2_mxfp8_4608x3072x9216": 43_854_336 + 42_894_336,   # gemm_pair_kernel<MXFP8, 256>
-}
+GEMM_TRAFFIC_BYTES = {}
 
 
 def _peaks():

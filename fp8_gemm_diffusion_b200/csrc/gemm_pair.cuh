@@ -13,23 +13,34 @@
 //   warp 0      A/B producer: each stage's 128 rows of A and BN/2 rows of B
 //               into this CTA's ring; completions land on the even CTA's full
 //               barrier (cta_group::2 loads, no multicast).
-//   warp 1      tensor memory (cta_group::2 allocation); on the even CTA one
-//               lane issues the MMAs and commits to both CTAs' barriers
-//               (multicast commit): stage free (its A/B slot and its scale
-//               set) and accumulator full.  A stage's commit is issued after
-//               the next stage's wait, so the wait never follows a commit.
+//   warp 1      tensor memory (cta_group::2 allocation); on the even CTA the
+//               converged warp runs the MMA loop and one elected lane issues
+//               each MMA and commit (descriptors and addresses stay
+//               warp-uniform).  Commits go to both CTAs' barriers (multicast
+//               commit): stage free (its A/B slot, and the scale set it used),
+//               right after the stage's MMAs, and accumulator full.  This
+//               warp never waits on a shared-memory barrier between MMAs: a
+//               shared-memory access right after a batch of MMAs stalls the
+//               issuing warp for a few hundred cycles, which left the tensor
+//               pipe idle once per stage.
+//   warp 3      stage waiter (even CTA): waits on the accumulator-empty and
+//               full barriers and hands each stage to warp 1 through a named
+//               barrier that also carries the "no timeout" flag.
 //   warp 2      scale loader: the scale chunks of each stage (A's 128 rows and
 //               all BN columns of B: each CTA's tensor memory needs B's) into
 //               a separate ring that runs ahead of the A/B ring.
 //   warps 4-7   scale writers, one per tensor-memory sub-partition: chunk rows
-//               from shared memory into the stage's set of tensor-memory
-//               columns with tcgen05.st, so no tcgen05.cp sits between MMAs;
-//               they arrive on the even CTA's full barrier of the stage, which
-//               thus completes when A, B and all scales are in place.
+//               from shared memory into a set of tensor-memory columns with
+//               tcgen05.st, so no tcgen05.cp sits between MMAs; they arrive on
+//               the even CTA's full barrier of the stage, which thus completes
+//               when A, B and all scales are in place.  The scale sets form
+//               their own ring (NSF <= STAGES sets, as many as tensor memory
+//               holds beside the accumulator), so the A/B ring can be deeper
+//               than the number of scale sets.
 //   warps 8-15  epilogue, sub-partition warp % 4, column half (warp / 4) % 2:
 //               the warp's accumulator columns into registers, release of the
-//               accumulator, then alpha, bias, bf16, 64-byte swizzled staging
-//               and TMA stores of 32 x 32 sub-tiles.
+//               accumulator, then alpha, bias, bf16, 32-byte swizzled staging
+//               (two buffers per warp) and TMA stores of 32 x 16 sub-tiles.
 // Tiles are visited along the smaller operand first (pair_tile_coords).
 // Every wait is bounded (ptx.cuh); a timed-out role stops, loads and MMAs in
 // flight are drained, and both CTAs free tensor memory together.
@@ -68,13 +79,13 @@ struct PairCfg {
   static constexpr uint32_t SF_TX = SFA_BYTES + SFB_BYTES;  // this CTA's scales
   static constexpr int SF_SLOT_BYTES = SCALED ? (SFA_BYTES + SFB_BYTES + 1023) / 1024 * 1024 : 0;
   static constexpr int SF_SLOTS = SCALED ? (F == Fmt::NVFP4 ? 4 : 8) : 0;
-  // tensor memory: the accumulator (BN columns), then one scale set per A/B
-  // stage (A chunks, then B chunks in MMA-major order, 4 columns each)
+  // tensor memory: the accumulator (BN columns), then the ring of scale sets
+  // (A chunks, then B chunks in MMA-major order, 4 columns each)
   static constexpr int SF_SET_COLS = (SF_CHUNKS + NRB * SF_CHUNKS) * 4;
   static constexpr int SF_COL = BN;
   static constexpr int SFB_OFF = SF_CHUNKS * 4;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int NS_FIT = SCALED ? (TMEM_COLS - BN) / SF_SET_COLS : 64;
+  static constexpr int NSF_FIT = SCALED ? (TMEM_COLS - BN) / SF_SET_COLS : 1;
   // warp roles, one warpgroup each for (producer, MMA, scale loader, spare),
   // the scale writers and the two halves of the epilogue
   static constexpr int SF_WARP0 = 4;   // warps 4-7, one per tensor-memory sub-partition
@@ -82,20 +93,24 @@ struct PairCfg {
   static constexpr int EPI_WARP0 = 8;  // warps 8-15: sub-partition warp % 4, column half (warp / 4) % 2
   static constexpr int EPI_WARPS = 8;
   static constexpr int EPI_COLS = BN / 2;   // accumulator columns per epilogue warp
-  static constexpr int EPI_SUB = 32;        // staging sub-tile: 32 rows x 32 columns (64-byte rows)
-  static constexpr int EPI_BYTES = EPI_WARPS * 32 * EPI_SUB * 2;
+  static constexpr int EPI_SUB = 16;        // staging sub-tile: 32 rows x 16 columns (32-byte rows)
+  static constexpr int EPI_BUFS = 2;        // per warp: fill one while the other is stored
+  static constexpr int EPI_BYTES = EPI_WARPS * EPI_BUFS * 32 * EPI_SUB * 2;
   // registers: launched with 65536 / 512 = 128 per thread, then rebalanced so
   // that an epilogue thread holds its 128 accumulator columns at once
   static constexpr int REGS_CTRL = 56, REGS_SFW = 80, REGS_EPI = 184;
   static constexpr int BAR_BYTES = 512;
   static constexpr int STAGES_FIT =
       (232448 - 1024 - BAR_BYTES - EPI_BYTES - SF_SLOTS * SF_SLOT_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES_MIN = STAGES_FIT < NS_FIT ? STAGES_FIT : NS_FIT;
-  static constexpr int STAGES = STAGES_MIN > 8 ? 8 : STAGES_MIN;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  // scale sets: as many as fit, at most one per A/B stage (a writer's wait for
+  // its set then also covers the stage's previous full-barrier phase)
+  static constexpr int NSF = SCALED ? (NSF_FIT < STAGES ? NSF_FIT : STAGES) : 1;
   // arrivals that complete a stage's full barrier besides the A/B bytes: the
   // producer's expect-tx and the scale writers of both CTAs
   static constexpr int FULL_ARRIVALS = 1 + (SCALED ? 2 * SF_WARPS : 0);
-  static_assert(STAGES >= 2, "shared / tensor memory");
+  static_assert(STAGES >= 2 && (!SCALED || NSF >= 2), "shared / tensor memory");
+  static_assert(4 * STAGES + 4 * SF_SLOTS + 32 <= BAR_BYTES / 4, "barrier area");
   static constexpr int SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + EPI_BYTES + BAR_BYTES;
   static constexpr int THREADS = 512;
@@ -129,6 +144,14 @@ __device__ __forceinline__ void pair_tile_coords(int tile, int m_tiles, int n_ti
     mt = tile - nt * m_tiles;
   }
 }
+
+// Named barrier between the MMA warp and the stage waiter (id 0 is __syncthreads).
+constexpr uint32_t kStageBar = 1;
+// MMA-issue order inside a stage: the next stage's handover goes before MMA
+// kHandoverBefore of the current one; with kLateCommit a stage's commit goes
+// behind the next stage's first MMA instead of right after its own MMAs.
+constexpr int kHandoverBefore = 3;
+constexpr bool kLateCommit = false;
 
 struct PairArgs {
   int M, N, K;
@@ -220,6 +243,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
   cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // B (the weight) is not the previous kernel's output: the B halves of the
+  // first stages are requested before the dependency wait, so that their
+  // latency overlaps that kernel's tail.  The producer below then issues only
+  // A for those stages.
+  const int a_row_off = static_cast<int>(rank) * C::BM_CTA;
+  const int b_row_off = static_cast<int>(rank) * C::BN_CTA;
+  constexpr int KX = C::ROW_BYTES / (F == Fmt::BF16 ? 2 : 1);  // K coordinate step per stage
+  const int n_pre = total_kb < S ? total_kb : S;                // stages with B requested early
+  if (warp == 0 && lane == 0) {
+    for (int g = 0; g < n_pre; ++g) {
+      const int tile = pair + (g / num_kb) * num_pairs, kb = g % num_kb;
+      int mt, nt;
+      pair_tile_coords(tile, m_tiles, n_tiles, n_fast, mt, nt);
+      if (rank == 0) mbar_arrive_expect_tx(full_bar(g), C::AB_PAIR_TX);
+      tma_load_2d_pair(base + g * C::STAGE_BYTES + C::A_BYTES, &tmap_b, map_to_cta(full_bar(g), 0),
+                       kb * KX, nt * BN + b_row_off);
+    }
+  }
   // everything above overlaps the previous kernel's tail; A, its scales and
   // the per-tensor scales are that kernel's output
   grid_dep_wait();
@@ -235,20 +276,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       int s = 0, issued = 0;
       uint32_t ph = 0;
       bool ok = true;
-      const int a_row_off = static_cast<int>(rank) * C::BM_CTA;
-      const int b_row_off = static_cast<int>(rank) * C::BN_CTA;
-      constexpr int KX = C::ROW_BYTES / (F == Fmt::BF16 ? 2 : 1);  // K coordinate step per stage
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
         int mt, nt;
         pair_tile_coords(tile, m_tiles, n_tiles, n_fast, mt, nt);
         const int a_row = mt * C::BM + a_row_off, b_row = nt * BN + b_row_off;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u)) { ok = false; break; }
-          if (rank == 0) mbar_arrive_expect_tx(full_bar(s), C::AB_PAIR_TX);
           const uint32_t leader_full = map_to_cta(full_bar(s), 0);
           const uint32_t sa = base + s * C::STAGE_BYTES;
+          if (issued >= n_pre) {
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(s), C::AB_PAIR_TX);
+            tma_load_2d_pair(sa + C::A_BYTES, &tmap_b, leader_full, kb * KX, b_row);
+          }
           tma_load_2d_pair(sa, &tmap_a, leader_full, kb * KX, a_row);
-          tma_load_2d_pair(sa + C::A_BYTES, &tmap_b, leader_full, kb * KX, b_row);
           ++issued;
           if (++s == S) { s = 0; ph ^= 1u; }
         }
@@ -263,10 +303,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // (one thread: keep the per-stage work to a few instructions)
-    if (lane == 0 && rank == 0) {
-      int s = 0, pend = -1;  // pend: stage whose MMAs are issued but not committed
-      uint32_t ph = 0, acc_ph = 0;
+    // The converged warp runs the loop (descriptors and addresses are
+    // warp-uniform); one elected lane issues each MMA and commit.  Stages
+    // arrive through the named barrier shared with the stage waiter (warp 3).
+    if (rank == 0) {
+      int s = 0, n = 0, pend = -1;  // A/B stage, scale set; pend: stage whose commit is deferred
       bool ok = true;
       const uint64_t adesc0 = desc_kmajor_sw128(base);
       const uint64_t bdesc0 = desc_kmajor_sw128(base + C::A_BYTES);
@@ -276,49 +317,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         int mt, nt;
         pair_tile_coords(tile, m_tiles, n_tiles, n_fast, mt, nt);
         const uint32_t sfb_shift = ((nt * BN) & 127) >> 5;
-        // the accumulator is single-buffered: wait until the epilogue has read the last tile
-        if (!mbar_wait_bounded(tempty_bar, acc_ph ^ 1u)) { ok = false; break; }
-        acc_ph ^= 1u;
-        tc_fence_after();
+        // the tile's first stage has landed and the accumulator is free
+        // (unless the waiter's bounded waits ran out)
+        if (!(ok = named_bar_and(kStageBar, 64, true))) break;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait_bounded(full_bar(s), ph)) { ok = false; break; }
-          // the previous stage's commit: after this wait, since a barrier wait
-          // issued right behind a commit takes a few hundred cycles longer
-          if (pend >= 0) tc_commit_pair(empty_bar(pend));
           tc_fence_after();
           const uint64_t adesc = adesc0 + DSTEP * s, bdesc = bdesc0 + DSTEP * s;
-          const uint32_t sf = tmem_base + C::SF_COL + s * C::SF_SET_COLS;
+          const uint32_t sf = tmem_base + C::SF_COL + n * C::SF_SET_COLS;
           int nmma = C::MMAS;
           if constexpr (F == Fmt::NVFP4) {
             if (kb == num_kb - 1) nmma = K / 64 - kb * C::MMAS;  // K % 256 != 0: partial last stage
           }
+          const bool next = kb + 1 < num_kb;  // then nmma == MMAS
 #pragma unroll
           for (int j = 0; j < C::MMAS; ++j) {
+            // The next stage's handover goes before this stage's last MMA: the
+            // handover stalls this warp until the MMAs issued so far are under
+            // way, and the last MMA still queued keeps the pipe busy meanwhile.
+            if (j == kHandoverBefore && next) ok = named_bar_and(kStageBar, 64, true);
             if (j < nmma) {
               const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
               const uint64_t koff = static_cast<uint64_t>(2 * j);  // 32 bytes of K per MMA
               if constexpr (F == Fmt::NVFP4) {
-                mma_pair_nvfp4(tmem_base, adesc + koff, bdesc + koff, idesc, sf + 4 * j,
-                               sf + C::SFB_OFF + j * C::NRB * 4 + sfb_shift, accum);
+                mma_pair_nvfp4_elect(tmem_base, adesc + koff, bdesc + koff, idesc, sf + 4 * j,
+                                     sf + C::SFB_OFF + j * C::NRB * 4 + sfb_shift, accum);
               } else if constexpr (F == Fmt::MXFP8) {
                 const uint32_t id = static_cast<uint32_t>(j) << 30;
-                mma_pair_mxfp8(tmem_base, adesc + koff, bdesc + koff,
-                               idesc | (static_cast<uint32_t>(j) << 4) | (static_cast<uint32_t>(j) << 29),
-                               sf | id, (sf + C::SFB_OFF + sfb_shift) | id, accum);
+                mma_pair_mxfp8_elect(tmem_base, adesc + koff, bdesc + koff,
+                                     idesc | (static_cast<uint32_t>(j) << 4) | (static_cast<uint32_t>(j) << 29),
+                                     sf | id, (sf + C::SFB_OFF + sfb_shift) | id, accum);
               } else {
-                mma_pair_bf16(tmem_base, adesc + koff, bdesc + koff, idesc, accum);
+                mma_pair_bf16_elect(tmem_base, adesc + koff, bdesc + koff, idesc, accum);
               }
             }
+            // a deferred commit of the previous stage, behind this stage's first MMA
+            if (kLateCommit && j == 0 && pend >= 0) {
+              tc_commit_pair_elect(empty_bar(pend));
+              pend = -1;
+            }
           }
-          pend = s;  // committed (A/B slot and scale set s free) after the next wait
-          if (++s == S) { s = 0; ph ^= 1u; }
+          if (kLateCommit) pend = s;                 // committed behind the next stage's first MMA
+          else tc_commit_pair_elect(empty_bar(s));   // A/B slot s and scale set n free once these complete
+          if (++s == S) s = 0;
+          if (++n == C::NSF) n = 0;
+          if (!ok) break;
         }
-        if (pend >= 0) tc_commit_pair(empty_bar(pend));
+        if (pend >= 0) tc_commit_pair_elect(empty_bar(pend));
         pend = -1;
         if (!ok) break;
-        tc_commit_pair(tfull_bar);
+        tc_commit_pair_elect(tfull_bar);
       }
-      tc_commit_pair(drain_bar);
+      tc_commit_pair_elect(drain_bar);
       mbar_wait_bounded(drain_bar, 0);
     } else if (lane == 0) {
       // odd CTA: the pair's MMAs read this CTA's memory; wait for the last one
@@ -358,7 +407,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       }
     }
   } else if (warp == 3) {
-    // spare warp of the control warpgroup
+    // ------------------------------------------------------------ stage waiter
+    // Waits, for the MMA warp, on the accumulator (once per tile) and on each
+    // stage's full barrier, then meets the MMA warp at the named barrier.  On
+    // a timeout it hands over "not ok" and both stop at the same handover.
+    if (rank == 0) {
+      int s = 0;
+      uint32_t ph = 0, acc_ph = 0;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        // the accumulator is single-buffered: the epilogue must have read the last tile
+        ok = mbar_wait_bounded(tempty_bar, acc_ph ^ 1u);
+        acc_ph ^= 1u;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          ok = ok && mbar_wait_bounded(full_bar(s), ph);
+          tc_fence_before();
+          named_bar_and(kStageBar, 64, ok);
+          if (!ok) break;
+          if (++s == S) { s = 0; ph ^= 1u; }
+        }
+      }
+    }
   }
   } else if (warp < C::EPI_WARP0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_SFW));
@@ -375,8 +444,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       const uint32_t leader_full0 = map_to_cta(full_bar(0), 0);
       constexpr int NA = C::SF_CHUNKS;            // A chunks per stage
       constexpr int NB = C::SF_CHUNKS * C::NRB;   // B chunks per stage
-      int r = 0, n = 0;
-      uint32_t rph = 0, nph = 0;
+      int r = 0, n = 0, s = 0;  // scale slot, scale set, A/B stage of g
+      int sp = 0;               // A/B stage of g - NSF (the last user of set n)
+      uint32_t rph = 0, spph = 0;
       for (int g = 0; g < total_kb; ++g) {
         if (!mbar_wait_bounded(sf_full_bar(r), rph)) break;
         const uint32_t slot = sf_base + r * C::SF_SLOT_BYTES;
@@ -392,10 +462,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
                        : "=r"(vb[4 * i]), "=r"(vb[4 * i + 1]), "=r"(vb[4 * i + 2]), "=r"(vb[4 * i + 3])
                        : "r"(slot + C::SFA_BYTES + (cb * C::SF_CHUNKS + jb) * 512 + lane * 16));
         }
-        // set n is free once the MMAs of stage g - S have completed; the full
-        // barrier of that stage has completed too, so the arrival below counts
-        // towards stage g
-        if (g >= S && !mbar_wait_bounded(empty_bar(n), nph ^ 1u)) break;
+        // set n is free once the MMAs of stage g - NSF (A/B stage sp) have
+        // completed.  NSF <= STAGES, so the full barrier of stage g - STAGES
+        // has completed too, and the arrival below counts towards stage g.
+        if (g >= C::NSF) {
+          if (!mbar_wait_bounded(empty_bar(sp), spph)) break;
+          if (++sp == S) { sp = 0; spph ^= 1u; }
+        }
         tc_fence_after();
         const uint32_t t = tmem_base + (q * 32u << 16) + C::SF_COL + n * C::SF_SET_COLS;
 #pragma unroll
@@ -422,11 +495,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         // before the warp's last loads had read the slot: a few lanes then
         // stored that stage's B scales for the last MMA of the stage.
         if (lane == 0) {
-          mbar_arrive_remote(leader_full0 + 8u * n);
+          mbar_arrive_remote(leader_full0 + 8u * s);
           mbar_arrive(sf_empty_bar(r));
         }
         if (++r == R) { r = 0; rph ^= 1u; }
-        if (++n == S) { n = 0; nph ^= 1u; }
+        if (++n == C::NSF) n = 0;
+        if (++s == S) s = 0;
       }
     }
   } else {
@@ -434,7 +508,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;          // tensor-memory sub-partition = 32-row slice
     const int h = (warp >> 2) & 1;   // column half of the tile
-    const uint32_t stage_buf = epi_base + (warp - C::EPI_WARP0) * (32 * C::EPI_SUB * 2);
+    const uint32_t stage_buf0 = epi_base + (warp - C::EPI_WARP0) * (C::EPI_BUFS * 32 * C::EPI_SUB * 2);
     const uint32_t leader_tempty = map_to_cta(tempty_bar, 0);
     float alpha = 1.0f;
     if constexpr (F == Fmt::NVFP4) alpha = (*args.a_g) * (*args.b_g);
@@ -479,11 +553,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       const int col_w = nt * BN + h * C::EPI_COLS;  // first column of this warp
 #pragma unroll
       for (int sub = 0; sub < C::EPI_COLS / C::EPI_SUB; ++sub) {
-        if (lane == 0) bulk_wait_group_read<0>();  // the staging sub-tile is free again
+        const uint32_t stage_buf = stage_buf0 + (sub & 1) * (32 * C::EPI_SUB * 2);
+        // this buffer's previous store (two sub-tiles ago) has read it
+        if (lane == 0) bulk_wait_group_read<C::EPI_BUFS - 1>();
         __syncwarp();
         // groups of 8 columns: alpha * acc + bias, bf16, one 16-byte store each
-        // into the 32 x EPI_SUB staging sub-tile (64 B rows, 64-byte swizzle:
-        // 16-byte chunk c of row l sits at chunk c ^ ((l / 2) % 4))
+        // into the 32 x EPI_SUB staging sub-tile (32 B rows, 32-byte swizzle:
+        // 16-byte chunk c of row l sits at chunk c ^ ((l / 4) % 2))
 #pragma unroll
         for (int j = 0; j < C::EPI_SUB / 8; ++j) {
           const int grp = h * (C::EPI_COLS / 8) + sub * (C::EPI_SUB / 8) + j;  // 8-column group in the tile
@@ -513,8 +589,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
             }
             pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
           }
-          static_assert(C::EPI_SUB == 32, "staging swizzle");
-          const uint32_t addr = stage_buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
+          static_assert(C::EPI_SUB == 16, "staging swizzle");
+          const uint32_t addr = stage_buf + lane * 32 + ((j ^ ((lane >> 2) & 1)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]),
                        "r"(pk[2]), "r"(pk[3])
                        : "memory");

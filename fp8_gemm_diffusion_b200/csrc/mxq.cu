@@ -356,7 +356,7 @@ mxq_status launch_gemm_pair(int dev, int sms, int slot, int64_t M, int64_t N, in
   }
   if (st == MXQ_OK)
     st = tmap_2d(&ty, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, ldy * 2, C::EPI_SUB, 32,
-                 CU_TENSOR_MAP_SWIZZLE_64B);
+                 CU_TENSOR_MAP_SWIZZLE_32B);  // 32 rows x 16 columns: 32-byte rows
   if (st != MXQ_OK) return st;
   mxq::PairArgs args;
   args.M = static_cast<int>(M);

@@ -62,9 +62,12 @@ def test_noalloc_matches_oracle_and_linear_on_two_calls_in_a_row(fmt):
     c = workloads.random_case(M, K, N, fmt, seed=31)
     w = mxq.Weight(c.W.to(DEV), c.bias.to(DEV), fmt=fmt)
     w.W_cpu = c.W
-    # two different activations: the second has a much smaller amax, so a
-    # stale amax or scale left in the scratch by the first call would show
-    inputs = [c.A, (c.A.float() * 1e-3).bfloat16()]
+    # two different activations: the second is the first times 2^-4 (exact in
+    # bf16), so its amax and every scale differ, and a stale amax or scale
+    # left in the scratch by the first call would show.  (A much smaller
+    # factor would make every output bias-dominated: the bf16 rounding of the
+    # bias alone then exceeds 2e-3 * sum|a b|, whose scale leaves the bias out.)
+    inputs = [c.A, (c.A.float() * 0.0625).bfloat16()]
     outs = []
     for a in inputs:
         y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
