@@ -39,8 +39,8 @@
 //               than the number of scale sets.
 //   warps 8-15  epilogue, sub-partition warp % 4, column half (warp / 4) % 2:
 //               the warp's accumulator columns into registers, release of the
-//               accumulator, then alpha, bias, bf16, 32-byte swizzled staging
-//               (two buffers per warp) and TMA stores of 32 x 16 sub-tiles.
+//               accumulator, then alpha, bias, bf16, swizzled staging (two
+//               buffers per warp) and TMA stores of 32 x EPI_SUB sub-tiles.
 // Tiles are visited along the smaller operand first (pair_tile_coords).
 // Every wait is bounded (ptx.cuh); a timed-out role stops, loads and MMAs in
 // flight are drained, and both CTAs free tensor memory together.
@@ -93,7 +93,8 @@ struct PairCfg {
   static constexpr int EPI_WARP0 = 8;  // warps 8-15: sub-partition warp % 4, column half (warp / 4) % 2
   static constexpr int EPI_WARPS = 8;
   static constexpr int EPI_COLS = BN / 2;   // accumulator columns per epilogue warp
-  static constexpr int EPI_SUB = 16;        // staging sub-tile: 32 rows x 16 columns (32-byte rows)
+  static constexpr int EPI_SUB = 32;        // staging sub-tile: 32 rows x EPI_SUB columns
+  static constexpr int EPI_ROW = EPI_SUB * 2;  // its row bytes, swizzled over the whole row (TMA swizzle mode)
   static constexpr int EPI_BUFS = 2;        // per warp: fill one while the other is stored
   static constexpr int EPI_BYTES = EPI_WARPS * EPI_BUFS * 32 * EPI_SUB * 2;
   // registers: launched with 65536 / 512 = 128 per thread, then rebalanced so
@@ -553,13 +554,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       const int col_w = nt * BN + h * C::EPI_COLS;  // first column of this warp
 #pragma unroll
       for (int sub = 0; sub < C::EPI_COLS / C::EPI_SUB; ++sub) {
-        const uint32_t stage_buf = stage_buf0 + (sub & 1) * (32 * C::EPI_SUB * 2);
+        const uint32_t stage_buf = stage_buf0 + (sub % C::EPI_BUFS) * (32 * C::EPI_SUB * 2);
         // this buffer's previous store (two sub-tiles ago) has read it
         if (lane == 0) bulk_wait_group_read<C::EPI_BUFS - 1>();
         __syncwarp();
         // groups of 8 columns: alpha * acc + bias, bf16, one 16-byte store each
-        // into the 32 x EPI_SUB staging sub-tile (32 B rows, 32-byte swizzle:
-        // 16-byte chunk c of row l sits at chunk c ^ ((l / 4) % 2))
+        // into the 32 x EPI_SUB staging sub-tile (EPI_ROW-byte rows, swizzled
+        // like the TMA's EPI_ROW-byte mode: 16-byte chunk c of row l sits at
+        // chunk c ^ ((l * EPI_ROW / 128) % (EPI_ROW / 16)))
 #pragma unroll
         for (int j = 0; j < C::EPI_SUB / 8; ++j) {
           const int grp = h * (C::EPI_COLS / 8) + sub * (C::EPI_SUB / 8) + j;  // 8-column group in the tile
@@ -589,8 +591,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
             }
             pk[e] = *reinterpret_cast<const uint32_t*>(&hv);
           }
-          static_assert(C::EPI_SUB == 16, "staging swizzle");
-          const uint32_t addr = stage_buf + lane * 32 + ((j ^ ((lane >> 2) & 1)) << 4);
+          static_assert(C::EPI_ROW == 32 || C::EPI_ROW == 64 || C::EPI_ROW == 128, "staging swizzle");
+          const uint32_t sw = (static_cast<uint32_t>(lane) * C::EPI_ROW / 128) & (C::EPI_ROW / 16 - 1);
+          const uint32_t addr = stage_buf + lane * C::EPI_ROW + ((j ^ sw) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]),
                        "r"(pk[2]), "r"(pk[3])
                        : "memory");

@@ -356,7 +356,8 @@ mxq_status launch_gemm_pair(int dev, int sms, int slot, int64_t M, int64_t N, in
   }
   if (st == MXQ_OK)
     st = tmap_2d(&ty, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, ldy * 2, C::EPI_SUB, 32,
-                 CU_TENSOR_MAP_SWIZZLE_32B);  // 32 rows x 16 columns: 32-byte rows
+                 C::EPI_ROW == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                  : (C::EPI_ROW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B));
   if (st != MXQ_OK) return st;
   mxq::PairArgs args;
   args.M = static_cast<int>(M);
@@ -445,13 +446,13 @@ bool valid_format(int f) { return f == MXQ_NVFP4 || f == MXQ_MXFP8 || f == MXQ_B
 // Byte layout of the weight storage and of the activation workspace:
 // [0,4) amax, [4,8) g, then (workspace only) the per-block amax partials at
 // [256, 256 + 4 * kMaxAmaxPartials), the single-pass quantiser's barrier
-// state (mxq::FusedSync, 256 bytes, then 8 bytes per CTA) from 4352, then
+// state (mxq::FusedSync, 256 bytes, then two 128-byte lines per CTA) from 4352, then
 // the codes and the scales, each 256-byte aligned.
 constexpr size_t kPartialsOff = 256;
 constexpr size_t kSyncOff = 4352;
-constexpr size_t kWorkspaceHeader = 8192;
+constexpr size_t kWorkspaceHeader = 4352 + 256 + 2 * 128 * 256 + 256;  // 70 KB
 static_assert(kPartialsOff + 4 * mxq::kMaxAmaxPartials <= kSyncOff, "workspace header");
-static_assert(kSyncOff + sizeof(mxq::FusedSync) + 8 * kFusedMaxGrid <= kWorkspaceHeader,
+static_assert(kSyncOff + sizeof(mxq::FusedSync) + 2 * 8 * mxq::kSyncLine * kFusedMaxGrid <= kWorkspaceHeader,
               "workspace header");
 struct QuantLayout {
   size_t codes_off, sf_off, total;

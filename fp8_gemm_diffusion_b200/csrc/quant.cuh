@@ -310,17 +310,21 @@ __global__ void __launch_bounds__(kQuantThreads)
 // once instead of twice, and one launch replaces two.
 //
 // Grid barrier, state in caller memory with any initial contents
-// (FusedSync below, then tags[grid]).  Every exchanged word is 64 bits,
-// written and read whole (single-copy atomic), so no fences are needed:
+// (FusedSync below, then tags[grid], then done[grid], one 128-byte line per
+// word, so that no line is polled by more than one CTA).  Every exchanged
+// word is 64 bits, written and read whole (single-copy atomic), so no fences
+// are needed:
 //   key     (epoch & 0xffff) << 48 | (~epoch & 0xffff) << 32, where epoch is
 //           read by every CTA at entry and advanced by CTA 0 once all CTAs
 //           have arrived (so no CTA reads the advanced value in the same
 //           launch).  Zeroed or byte-filled memory never matches a key (its
 //           two halves are not complements);
 //   tags[b] key | bits(maximum of CTA b), its arrival;
-//   done    key | bits(amax): CTA 0 waits for every tag, publishes done and
-//           clears the tags; every CTA waits on that one word, so the polling
-//           stays off the tag lines.
+//   done[b] key | bits(amax), CTA b's copy of the result: CTA 0 waits for
+//           every tag, writes every CTA's copy and clears the tags; CTA b
+//           waits on its own copy and clears it once read.  (With every CTA
+//           on one shared word, and the tags packed into a few lines, the
+//           polling itself slowed the exchange to several microseconds.)
 // The launch is cooperative (all CTAs resident together) and every wait is
 // bounded: on timeout the CTA records kErrTimeout and leaves its rows
 // unquantised (CTA 0 still advances the epoch, so a later launch never
@@ -328,7 +332,9 @@ __global__ void __launch_bounds__(kQuantThreads)
 constexpr int kFusedThreads = 1024;
 constexpr int kFusedWarps = kFusedThreads / 32;
 
-struct FusedSync {                 // 256 bytes, then tags[grid]
+constexpr int kSyncLine = 16;      // 64-bit words per 128-byte line
+
+struct FusedSync {                 // 256 bytes, then tags[grid] and done[grid], a line each
   unsigned int epoch;
   unsigned int pad0;
   unsigned long long done;
@@ -391,6 +397,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const int nr = min(rows_per_cta, rows - r0);
   const int vpr = k >> 3;  // 16-byte vectors per row
   unsigned long long* const tags = reinterpret_cast<unsigned long long*>(sync + 1);
+  unsigned long long* const done = tags + static_cast<size_t>(gridDim.x) * kSyncLine;
 
   grid_dep_wait();  // x is the previous kernel's output
   if (threadIdx.x == 0) {
@@ -428,7 +435,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   if (warp == 0) {
     float b = lane < kFusedWarps ? s_red[lane] : 0.0f;
     b = warp_max(b);
-    if (lane == 0) st_relaxed_u64(tags + blockIdx.x, key | __float_as_uint(b));
+    if (lane == 0) st_relaxed_u64(tags + blockIdx.x * kSyncLine, key | __float_as_uint(b));
     __syncwarp();
     bool ok = true;
     if (blockIdx.x == 0) {
@@ -439,7 +446,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         bool mine = true;
         a = 0.0f;
         for (int c = lane; c < nb; c += 32) {
-          const unsigned long long w = ld_relaxed_u64(tags + c);
+          const unsigned long long w = ld_relaxed_u64(tags + c * kSyncLine);
           mine &= (w & kKeyMask) == key;
           a = fmaxf(a, __uint_as_float(static_cast<uint32_t>(w)));
         }
@@ -450,15 +457,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         }
       }
       a = warp_max(a);
-      if (ok && lane == 0) st_relaxed_u64(&sync->done, key | __float_as_uint(a));
-      for (int c = lane; c < nb; c += 32) st_relaxed_u64(tags + c, 0ull);
+      for (int c = lane; c < nb; c += 32) {
+        if (ok) st_relaxed_u64(done + c * kSyncLine, key | __float_as_uint(a));
+        st_relaxed_u64(tags + c * kSyncLine, 0ull);
+      }
       if (lane == 0) sync->epoch = s_epoch + 1u;  // every CTA read the epoch before its tag
     }
     if (lane == 0) {
       uint32_t bits = 0;
-      ok = ok && spin_for_key(&sync->done, key, bits);
-      if (ok) s_amax = __uint_as_float(bits);
-      else record_error(kErrTimeout);
+      ok = ok && spin_for_key(done + blockIdx.x * kSyncLine, key, bits);
+      if (ok) {
+        s_amax = __uint_as_float(bits);
+        st_relaxed_u64(done + blockIdx.x * kSyncLine, 0ull);  // read: cleared for later launches
+      } else {
+        record_error(kErrTimeout);
+      }
       s_ok = ok ? 1 : 0;
     }
   }

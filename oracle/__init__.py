@@ -15,6 +15,8 @@ Plain numpy, written to be checked by eye against the definitions:
 * ``dispatch`` - the selective-quantisation rule.
 * ``producer`` - a linear layer with the GELU activation fused into its
   epilogue, and that epilogue's error scale.
+* ``attention`` - 8-bit (MXFP8) attention with per-token scales: softmax in
+  float64 on the dequantised operands, and its error bound.
 
 Every function is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle_*.py`` to facts other than itself (code tables, tie cases,
@@ -23,7 +25,7 @@ cast, byte offsets of the scale-factor layout worked by hand from its
 published description).
 """
 
-from . import formats, quant, gemm, dispatch, producer  # noqa: F401
+from . import formats, quant, gemm, dispatch, producer, attention  # noqa: F401
 from .formats import *  # noqa: F401,F403
 from .quant import *  # noqa: F401,F403
 from .gemm import *  # noqa: F401,F403

@@ -24,8 +24,19 @@ import fp8_gemm_diffusion_b200 as mxq
 
 pytestmark = pytest.mark.gpu
 
-HEADER = 8192          # workspace header: amax, g, amax partials, barrier state
 SMEM_LIMIT = 227 * 1024 - 1024
+
+
+def _pad256(n):
+    return (n + 255) // 256 * 256
+
+
+def _header(M, K):
+    """Bytes before the codes in the workspace (amax, g, amax partials,
+    barrier state): the workspace is header + codes + scales, each part
+    padded to 256 bytes."""
+    return (mxq.linear_workspace_bytes(M, K, "nvfp4") - _pad256(M * K // 2)
+            - _pad256(Q.sf_bytes(M, K, 16)))
 
 
 def _single_pass(M, K):
@@ -58,6 +69,8 @@ def _check(ws, A):
     assert float(amax) == float(oq["amax"]), "amax"
     assert g == oq["g"], "per-tensor scale g"
     nc = M * K // 2
+    HEADER = _header(M, K)
+    assert HEADER % 256 == 0 and HEADER >= 8
     codes = st[HEADER: HEADER + nc].reshape(M, K // 2)
     bad = np.argwhere(codes != oq["codes"])
     assert bad.size == 0, f"{len(bad)} code bytes differ, first at {bad[:4].tolist()}"
