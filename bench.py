@@ -657,6 +657,119 @@ def run_stack(args, rank, world, local_rank):
     }
 
 
+# ------------------------------------------------------------- attention
+def run_attention(args, rank, world, local_rank):
+    """One step = one FLUX-shaped attention (24 heads x 4608 tokens x 128)
+    through mxq_attention_mxfp8: per-token MXFP8 of Q and K, MXFP8 of V^T,
+    then the attention kernel.  The metric counts the attention's two
+    products, 4 * heads * tokens^2 * d per step (the kernel runs the first
+    product twice, once per softmax pass: 6 * heads * tokens^2 * d on the
+    tensor cores, which the roofline uses).  Baseline: PyTorch's
+    scaled_dot_product_attention in bf16 on the same tensors."""
+    import torch.nn.functional as Fn
+
+    import fp8_gemm_diffusion_b200 as mxq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    H, T, d = 24, 4608, 128
+    Q, K, V = (t.to(dev) for t in workloads.flux_attention(H, T, d))
+    nsets = 4  # 4 x 85 MB of inputs rotate: no step starts with its inputs in L2
+    sets = [(Q.clone(), K.clone(), V.clone(), torch.empty_like(Q)) for _ in range(nsets)]
+    nbytes = mxq.attention_workspace_bytes(H, T, d)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    flops = 4.0 * H * T * T * d
+    mma_flops = 6.0 * H * T * T * d
+
+    def step(i):
+        q, k, v, o = sets[i % nsets]
+        mxq.attention_mxfp8(q, k, v, H, T, o, ws, nbytes, stream=stream)
+
+    def timed(fn, n):
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.barrier()
+        torch.cuda.synchronize()
+        torch.cuda._sleep(SPIN_CYCLES)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), dev)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if mxq.get_device_error() != mxq.OK:
+        raise RuntimeError("device-side timeout during warm-up")
+    sampler = ClockSampler(_nvml_id(local_rank))
+    sampler.start()
+    t0 = time.perf_counter()
+    total_ms = timed(step, args.steps)
+    sampler.mark("headline", t0, time.perf_counter())
+    # the attention kernel alone (the quantisers' share is the rest of the step)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+    for i, (a, b) in enumerate(evs):
+        q, k, v, o = sets[i % nsets]
+        a.record(stream)
+        step(i)
+        b.record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    call_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    if mxq.get_device_error() != mxq.OK:
+        raise RuntimeError("device-side timeout during the timed steps")
+
+    def sdpa(i):
+        q, k, v, o = sets[i % nsets]
+        o.copy_(Fn.scaled_dot_product_attention(q.unsqueeze(0), k.unsqueeze(0), v.unsqueeze(0))[0])
+
+    for i in range(args.warmup):
+        sdpa(i)
+    bf16_ms = timed(sdpa, max(1, min(args.steps, 50))) / max(1, min(args.steps, 50))
+    step_ms = total_ms / args.steps
+    value = whole_job_tflops(world, 1, flops, step_ms)
+    peaks = _peaks()
+    peak = peaks["bf16"] * NOMINAL_RATIO["mxfp8"]
+    return {
+        "metric": "8-bit attention TFLOPS incl. quantisation (4 H T^2 d per step)",
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3+e8m0 (mxfp8) Q, K, V and softmax weights; fp32 softmax and accumulate; bf16 out",
+        "data": "synthetic (seeded FLUX-shaped Q, K, V ~ N(0, 1))",
+        "config": {"workload": f"flux_attention_{H}x{T}x{d}", "heads": H, "tokens": T, "head_dim": d,
+                   "parallelism": f"replicas x{world}",
+                   "step": "mxq_attention_mxfp8: MXFP8 of Q, K (per token) and V^T, two-pass softmax attention",
+                   "l2": f"rotating {nsets} input sets ({nsets * 4 * H * T * d * 2 / 2**20:.0f} MiB > 126 MiB L2)"},
+        "kernels_ms": {"step": round(step_ms, 5), "call_with_events": round(call_ms, 5)},
+        "roofline": {"kernel": "attention_mxfp8_kernel + quantisers", "bound": "tensor",
+                     "achieved": round(mma_flops / (step_ms * 1e-3) / 1e12, 2), "peak": round(peak, 1),
+                     "unit": "TFLOP/s", "frac": round(mma_flops / (step_ms * 1e-3) / 1e12 / peak, 4),
+                     "peak_kind": "burst",
+                     "peak_source": f"{peaks['source']} bf16 burst x 2 (nominal fp8:bf16 dense ratio); "
+                                    "achieved counts the 6 H T^2 d tensor-core flops the kernel runs",
+                     "traffic": None},
+        "bf16_baseline": {"impl": "torch scaled_dot_product_attention, bf16, same tensors",
+                          "value": round(whole_job_tflops(world, 1, flops, bf16_ms), 2), "unit": UNIT,
+                          "ms_per_step": round(bf16_ms, 5), "speedup_of_value": round(bf16_ms / step_ms, 3)},
+        "clocks": sampler.summary("headline"),
+        "e2e": None,
+        "gpu_launches": 4 * args.steps,
+        "cpu_baseline": None,
+    }
+
+
 # ------------------------------------------------------------- CPU oracle
 def run_oracle_sample(workload: str, budget_s: float = 12.0):
     """Time the oracle (as it stands) on a bounded sample of the workload:
@@ -712,7 +825,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5", "attn"])
     ap.add_argument("--batch", type=int, default=1, choices=[1, 4],
                     help="batch of the c5 stack (1: 4608 tokens per image)")
     ap.add_argument("--impl", default="mxq", choices=["mxq", "reference"])
@@ -735,9 +848,9 @@ def main():
         # the CPU oracle on the host cores: rank 0 only, a few bounded samples
         if rank != 0:
             return 0
-        if args.workload == "c5":
+        if args.workload in ("c5", "attn"):
             print(json.dumps({"impl": "reference", "unavailable": "the oracle arm times single "
-                              "layers (c1-c4); the c5 stack is a sequence of those layers"}))
+                              "linear layers (c1-c4)"}))
             return 0
         steps = max(1, min(args.steps, 3))
         per_step, sample = [], None
@@ -767,8 +880,8 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device("cuda", local_rank))
     try:
-        if args.workload == "c5":
-            result = run_stack(args, rank, world, local_rank)
+        if args.workload in ("c5", "attn"):
+            result = (run_stack if args.workload == "c5" else run_attention)(args, rank, world, local_rank)
             if rank == 0:
                 print(json.dumps(result))
             return 0

@@ -113,6 +113,9 @@ _linear_noalloc = _proto("mxq_linear_noalloc", _int, ctypes.POINTER(mxq_weight),
 _linear_kernel_count = _proto("mxq_linear_kernel_count", _int, ctypes.POINTER(mxq_weight), _i64,
                               ctypes.POINTER(mxq_linear_opts))
 _get_device_error = _proto("mxq_get_device_error", _int, _ptr)
+_attention_workspace_bytes = _proto("mxq_attention_workspace_bytes", _sz, _i64, _i64, _i64)
+_attention_mxfp8 = _proto("mxq_attention_mxfp8", _int, _ptr, _ptr, _ptr, _i64, _i64, _i64, ctypes.c_float,
+                          _ptr, _ptr, _sz, _ptr)
 _convert_f32 = _proto("mxq_convert_f32", _int, _ptr, _i64, _int, _ptr, _ptr)
 
 #: Every symbol include/mxq.h declares (checked by the CPU tests).
@@ -122,6 +125,7 @@ EXPORTED = [
     "mxq_gemm_blockscaled", "mxq_weight_storage_bytes", "mxq_weight_prepare",
     "mxq_linear_path", "mxq_linear_workspace_bytes", "mxq_linear", "mxq_get_device_error",
     "mxq_convert_f32", "mxq_linear_noalloc", "mxq_linear_kernel_count", "mxq_quantize_mxfp8_rule",
+    "mxq_attention_workspace_bytes", "mxq_attention_mxfp8",
 ]
 
 #: Capacity of the static device scratch of mxq_linear_noalloc (MXQ_NOALLOC_SCRATCH_BYTES).
@@ -286,6 +290,28 @@ def linear_noalloc(w: mxq_weight, x, M, y, min_dim=None, stream=None) -> None:
     instead.  Calls that overlap on the GPU race on that shared scratch."""
     _check(_linear_noalloc(ctypes.byref(w), _addr(x), M, _addr(y), _opts(min_dim),
                            _stream(stream)), "mxq_linear_noalloc")
+
+
+def attention_workspace_bytes(heads: int, tokens: int, d: int = 128) -> int:
+    return _attention_workspace_bytes(heads, tokens, d)
+
+
+def attention_mxfp8(q, k, v, heads, tokens, out, ws, ws_bytes, d=128, tau=0.0, stream=None) -> None:
+    """out = attention(q, k, v) per head through the 8-bit path; q, k, v, out
+    [heads][tokens][d] bf16 (tensors or device addresses)."""
+    _check(_attention_mxfp8(_addr(q), _addr(k), _addr(v), heads, tokens, d, float(tau), _addr(out),
+                            _addr(ws), ws_bytes, _stream(stream)), "mxq_attention_mxfp8")
+
+
+def attention_forward(q, k, v, tau=0.0, stream=None):
+    """Allocates the output and workspace with torch; q, k, v [heads, tokens, d] bf16."""
+    import torch
+    H, T, d = q.shape
+    out = torch.empty_like(q)
+    nbytes = attention_workspace_bytes(H, T, d)
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    attention_mxfp8(q, k, v, H, T, out, ws, nbytes, d=d, tau=tau, stream=stream)
+    return out
 
 
 def get_device_error(stream=None) -> int:

@@ -93,9 +93,9 @@ struct PairCfg {
   static constexpr int EPI_WARP0 = 8;  // warps 8-15: sub-partition warp % 4, column half (warp / 4) % 2
   static constexpr int EPI_WARPS = 8;
   static constexpr int EPI_COLS = BN / 2;   // accumulator columns per epilogue warp
-  static constexpr int EPI_SUB = 32;        // staging sub-tile: 32 rows x EPI_SUB columns
+  static constexpr int EPI_SUB = 16;        // staging sub-tile: 32 rows x EPI_SUB columns
   static constexpr int EPI_ROW = EPI_SUB * 2;  // its row bytes, swizzled over the whole row (TMA swizzle mode)
-  static constexpr int EPI_BUFS = 2;        // per warp: fill one while the other is stored
+  static constexpr int EPI_BUFS = 1;        // per warp (a second buffer measured no faster and costs a stage)
   static constexpr int EPI_BYTES = EPI_WARPS * EPI_BUFS * 32 * EPI_SUB * 2;
   // registers: launched with 65536 / 512 = 128 per thread, then rebalanced so
   // that an epilogue thread holds its 128 accumulator columns at once

@@ -17,6 +17,7 @@
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "quant.cuh"
+#include "attention.cuh"
 
 namespace {
 
@@ -465,6 +466,27 @@ QuantLayout quant_layout(int64_t rows, int64_t k, mxq_format f, size_t header = 
   return l;
 }
 
+// Byte layout of the attention workspace: MXFP8 codes and scales of Q and K
+// (rows heads * tokens, 128 channels) and of V^T (rows heads * 128, tokens),
+// each part 256-byte aligned.
+struct AttLayout {
+  size_t q_codes, q_sf, k_codes, k_sf, v_codes, v_sf, total;
+};
+AttLayout att_layout(int64_t heads, int64_t tokens) {
+  AttLayout l;
+  const int64_t rows = heads * tokens, vrows = heads * mxq::kAttD;
+  size_t off = 0;
+  auto take = [&](size_t n) { const size_t o = off; off += static_cast<size_t>(pad_to(static_cast<int64_t>(n), 256)); return o; };
+  l.q_codes = take(static_cast<size_t>(rows) * mxq::kAttD);
+  l.q_sf = take(mxq_sf_bytes(rows, mxq::kAttD, MXQ_MXFP8));
+  l.k_codes = take(static_cast<size_t>(rows) * mxq::kAttD);
+  l.k_sf = take(mxq_sf_bytes(rows, mxq::kAttD, MXQ_MXFP8));
+  l.v_codes = take(static_cast<size_t>(vrows) * tokens);
+  l.v_sf = take(mxq_sf_bytes(vrows, tokens, MXQ_MXFP8));
+  l.total = off;
+  return l;
+}
+
 }  // namespace
 
 // =====================================================================  ABI
@@ -808,6 +830,70 @@ int mxq_linear_kernel_count(const mxq_weight* w, int64_t M, const mxq_linear_opt
   int dev, sms;
   if (current_device(&dev, &sms) != MXQ_OK) return -1;
   return plan_fused(M, w->K, sms).grid > 0 ? 2 : 3;
+}
+
+size_t mxq_attention_workspace_bytes(int64_t heads, int64_t tokens, int64_t d) {
+  if (heads <= 0 || tokens <= 0 || d != mxq::kAttD) return 0;
+  return att_layout(heads, tokens).total;
+}
+
+mxq_status mxq_attention_mxfp8(const void* q, const void* k, const void* v, int64_t heads,
+                               int64_t tokens, int64_t d, float tau, void* out, void* ws,
+                               size_t ws_bytes, mxq_stream_t stream) {
+  if (heads < 0 || tokens < 0) return MXQ_ERR_INVALID_ARG;
+  if (d != mxq::kAttD) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  if (heads == 0 || tokens == 0) return MXQ_OK;
+  if (tokens % mxq::kAttTile != 0) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  if (heads * tokens > INT32_MAX / 2 || heads * tokens * d > (int64_t(1) << 40)) return MXQ_ERR_UNSUPPORTED_SHAPE;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || ws == nullptr) return MXQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MXQ_ERR_ALIGNMENT;
+  if (!aligned256(ws)) return MXQ_ERR_ALIGNMENT;
+  const AttLayout l = att_layout(heads, tokens);
+  if (ws_bytes < l.total) return MXQ_ERR_WORKSPACE;
+  if (!(tau > 0.0f) || !(tau < INFINITY)) tau = 1.0f / sqrtf(static_cast<float>(d));
+  int dev, sms;
+  mxq_status st;
+  if ((st = current_device(&dev, &sms)) != MXQ_OK) return st;
+  if ((st = get_encoder()) != MXQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const int64_t rows = heads * tokens;
+  // per-token MXFP8 of Q and K (rows of 128 channels), V^T along tokens
+  if ((st = launch_quant_mxfp8(q, rows, d, d, base + l.q_codes, base + l.q_sf, s, sms)) != MXQ_OK) return st;
+  if ((st = launch_quant_mxfp8(k, rows, d, d, base + l.k_codes, base + l.k_sf, s, sms)) != MXQ_OK) return st;
+  const int grid = static_cast<int>(heads * (tokens / mxq::kAttTile));
+  cudaError_t e = launch_pdl(mxq::quantize_mxfp8_vt_kernel, dim3(grid), dim3(512), 0, s,
+                             static_cast<const __nv_bfloat16*>(v), static_cast<int>(heads),
+                             static_cast<int>(tokens), base + l.v_codes, base + l.v_sf);
+  if (e != cudaSuccess) return cuda_fail(e);
+  constexpr uint32_t bit = 1u << 21;  // GEMM instantiations and the fused quantiser use lower bits
+  if (!(g_dev[dev].smem_attr_set.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(mxq::attention_mxfp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             mxq::AttCfg::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_dev[dev].smem_attr_set.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  CUtensorMap tq, tk, tv;
+  if ((st = tmap_2d(&tq, base + l.q_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d, rows, d, 128, mxq::kAttTile,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != MXQ_OK)
+    return st;
+  if ((st = tmap_2d(&tk, base + l.k_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, d, rows, d, 128, mxq::kAttTile,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != MXQ_OK)
+    return st;
+  if ((st = tmap_2d(&tv, base + l.v_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, tokens, heads * d, tokens, 128,
+                    mxq::kAttD, CU_TENSOR_MAP_SWIZZLE_128B)) != MXQ_OK)
+    return st;
+  mxq::AttArgs args;
+  args.heads = static_cast<int>(heads);
+  args.tokens = static_cast<int>(tokens);
+  args.c = tau * 1.4426950408889634f;  // tau * log2(e): the weights are powers of two
+  args.q_sf = base + l.q_sf;
+  args.k_sf = base + l.k_sf;
+  args.v_sf = base + l.v_sf;
+  args.out = static_cast<__nv_bfloat16*>(out);
+  e = launch_pdl(mxq::attention_mxfp8_kernel, dim3(grid), dim3(mxq::AttCfg::THREADS), mxq::AttCfg::SMEM_BYTES, s,
+                 tq, tk, tv, args);
+  return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
 mxq_status mxq_get_device_error(mxq_stream_t stream) {

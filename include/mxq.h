@@ -305,6 +305,48 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
 mxq_status mxq_linear_noalloc(const mxq_weight* w, const void* x_bf16, int64_t M, void* y_bf16,
                               const mxq_linear_opts* opts, mxq_stream_t stream);
 
+/* ------------------------------------------------------- attention ----- */
+
+/*
+ * 8-bit attention with per-token scales (the devin.kr page on Blackwell FLUX
+ * image generation, "엔비디아 블랙웰 기반 플럭스 3 이미지 생성 4.45배 가속",
+ * section "연산 효율화와 가속 기술": a dedicated 8-bit floating-point attention
+ * path that corrects the quantisation error token by token).  Per head, with
+ * T tokens and head dimension d = 128:
+ *   Q, K -> MXFP8 (E4M3 codes, one power-of-two scale per token and per 32
+ *   channels), V -> MXFP8 of V^T (per channel and per 32 tokens);
+ *   S = deq(Q) deq(K)^T on the tensor cores (fp32); softmax along keys with
+ *   scale tau, exact (row maximum first, then the weights
+ *   E = 2^((S - max) tau log2 e) in fp32); E -> MXFP8 along keys (ceiling
+ *   scale rule, no saturation); O = deq(E) deq(V^T)^T / rowsum(E) on the
+ *   tensor cores (fp32), bf16 out.
+ * Accuracy: |O - O_exact| <= 0.07 * T + 1e-6 per element, with O_exact the
+ * float64 attention on the quantised Q, K, V and T = sum over 32-key blocks
+ * of (the block's softmax mass) x (the block's max |V|) -- the rounding of E
+ * to E4M3 (at most 2^-4 of each weight) dominates.
+ *
+ * mxq_attention_workspace_bytes - device bytes mxq_attention_mxfp8 needs
+ * (the quantised Q, K, V^T and their scales); 0 for unsupported arguments.
+ */
+size_t mxq_attention_workspace_bytes(int64_t heads, int64_t tokens, int64_t d);
+
+/*
+ * mxq_attention_mxfp8 - out = attention(q, k, v) per head.
+ *   q, k, v, out: [heads][tokens][d] bf16, contiguous, device, 16-byte aligned.
+ *   d must be 128 and tokens a multiple of 128 (else UNSUPPORTED_SHAPE).
+ *   tau: softmax scale; 0 (or any non-positive or non-finite value) means
+ *   1/sqrt(d).
+ *   ws: device workspace of mxq_attention_workspace_bytes(heads, tokens, d)
+ *   bytes, 256-byte aligned; any contents on entry.
+ * Four launches on `stream` (Q and K quantisation, V^T quantisation, the
+ * attention kernel), no host synchronisation, nothing allocated.  Argument
+ * errors return before anything is enqueued; device-side timeouts show in
+ * mxq_get_device_error.  Calls sharing a workspace must be ordered on the GPU.
+ */
+mxq_status mxq_attention_mxfp8(const void* q_bf16, const void* k_bf16, const void* v_bf16,
+                               int64_t heads, int64_t tokens, int64_t d, float tau, void* out_bf16,
+                               void* ws, size_t ws_bytes, mxq_stream_t stream);
+
 /* ---------------------------------------------------- diagnostics ------- */
 
 /*

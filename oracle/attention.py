@@ -19,27 +19,40 @@ MXFP8" on the B200 MXFP8/NVFP4 diffusion article):
      second product's contraction (over tokens) sees one scale per 32 terms;
   3. S = tau * deq(Qq) deq(Kq)^T, tau = 1 / sqrt(d);
   4. P = softmax(S) along keys (exact: maximum subtracted, normalised);
-  5. the kernel quantises P (in fp32) to MXFP8 along keys and computes
-     O = deq(Pq) deq(Vq)^T with fp32 accumulation, bf16 output.
+  5. the kernel quantises the unnormalised weights E = exp(S - rowmax(S)),
+     in [0, 1] and in fp32, to MXFP8 along keys with the ceiling scale rule
+     (the smallest shared exponent with no saturation: under the floor rule
+     a block maximum in [448, 512) * 2^X would be clipped to 448, up to
+     12.5 % off), computes deq(Eq) deq(Vq)^T with fp32 accumulation and
+     divides by the row sum of E (fp32); bf16 output.
 
 The oracle evaluates steps 1-4 exactly (float64 after the quantisers) and
 O_ref = P deq(Vq)^T without rounding P.  The error of step 5 is bounded by
-the rounding of P: E4M3 keeps 3 fraction bits, so a normal value moves by at
-most 2^-4 of itself; values below the block's normal range (E4M3 subnormals
-and zero) move by at most 2^-10 of the block scale, i.e. 2^-18 of the block
-maximum, which is at most the block's sum.  With the block-wise error scale
+the rounding of E (relative errors carry over to P = E / sum E): E4M3 keeps
+3 fraction bits, so a normal value moves by at most 2^-4 of itself (nothing
+saturates under the ceiling rule); values below the block's normal range
+(E4M3 subnormals and zero) move by at most 2^-10 of the block scale, i.e. at
+most 2^-17 of the block maximum (the ceiling rule puts the maximum at
+224 * 2^X or above), which is at most the block's sum.  With the error scale
 
-  T[i, c] = sum_b ( sum_{j in b} P[i, j] ) * max_{j in b} |deq(Vq)^T[j, c]|
+  T[i, c] = sum_j P[i, j] |deq(Vq)^T[j, c]|      (T >= |O[i, c]|)
 
-(b running over blocks of 32 keys; T >= sum_j P[i, j] |V[j, c]| >= |O[i, c]|)
-the rounding of P contributes at most (2^-4 + 32 * 2^-18) T, the bf16
-output 2^-9 T, fp32 accumulation and the fp32 exponential far less, so
+the normal-range rounding contributes at most 2^-4 T; the underflowed
+weights at most 32 * 2^-17 of each block's sum times that block's largest
+|V|, in all at most 2^-12 max_j |V[j, c]|; the bf16 output 2^-9 T; fp32
+accumulation and the fp32 exponential far less.  So every element satisfies
 
-  |O_gpu - O_ref| <= ATT_RTOL * T + ATT_ATOL,  ATT_RTOL = 0.07, ATT_ATOL = 1e-6.
+  |O_gpu - O_ref| <= ATT_RTOL * T + 2^-12 * max_j |V[j, c]| + ATT_ATOL,
+  ATT_RTOL = 0.07, ATT_ATOL = 1e-6                       (within_att_tol)
 
-``attention_ref`` also returns O_q, the product with P quantised by the
-oracle's own MXFP8 quantiser (P rounded to fp32 first): the kernel differs
-from it only where its fp32 P falls on the other side of a rounding boundary.
+This worst case is loose when the weights are spread over many keys.  The
+sharp check is against O_q, step 5 done by the oracle: E rounded to fp32 and
+quantised by its own MXFP8 quantiser (ceiling rule), the product in float64,
+divided by the float64 row sum of E.  The kernel differs from it only where
+its fp32 E falls on the other side of a rounding boundary (a weight moves by
+one E4M3 step) and by fp32 accumulation and the bf16 output, so nearly every
+element satisfies the GEMM's rule |O_gpu - O_q| <= 2e-3 T + 1e-6
+(within_att_tight).
 """
 
 from __future__ import annotations
@@ -50,7 +63,8 @@ import numpy as np
 
 from .quant import _as_f32, dequant_mxfp8, quantize_mxfp8
 
-__all__ = ["softmax_rows", "attention_plain", "attention_ref", "ATT_RTOL", "ATT_ATOL", "within_att_tol"]
+__all__ = ["softmax_rows", "attention_plain", "attention_ref", "ATT_RTOL", "ATT_ATOL", "within_att_tol",
+           "within_att_tight"]
 
 ATT_RTOL = 0.07
 ATT_ATOL = 1e-6
@@ -80,8 +94,8 @@ def attention_ref(Q, K, V, rows=None, tau=None):
 
     Q, K, V: [T, d] (torch bf16 tensors or float32 arrays), T and d multiples
     of 32.  rows: optional query rows to evaluate (the quantisation of K and
-    V always uses every token).  Returns (O_ref, T_err, O_q), each [rows, d]
-    float64.
+    V always uses every token).  Returns (O_ref, T_err, O_q, vmax): the
+    first three [rows, d] float64, vmax [d] = max_j |deq(Vq)^T[j, c]|.
     """
     Qf, Kf, Vf = _as_f32(Q), _as_f32(K), _as_f32(V)
     T_, d = Qf.shape
@@ -97,16 +111,25 @@ def attention_ref(Q, K, V, rows=None, tau=None):
     Vd = dequant_mxfp8(vq["codes"], vq["sf"]).T          # [T, d]
     P = softmax_rows(tau * (Qd @ Kd.T))                   # [rows, T]
     O = P @ Vd
-    nb = T_ // KEY_BLOCK
-    Pb = P.reshape(P.shape[0], nb, KEY_BLOCK).sum(axis=2)             # [rows, nb]
-    Vb = np.abs(Vd).reshape(nb, KEY_BLOCK, d).max(axis=1)             # [nb, d]
-    T_err = Pb @ Vb
-    pq = quantize_mxfp8(P.astype(np.float32))
-    Oq = dequant_mxfp8(pq["codes"], pq["sf"]) @ Vd
-    return O, T_err, Oq
+    T_err = P @ np.abs(Vd)
+    vmax = np.abs(Vd).max(axis=0)
+    S = tau * (Qd @ Kd.T)
+    E = np.exp(S - S.max(axis=1, keepdims=True))
+    eq = quantize_mxfp8(E.astype(np.float32), scale_rule="rceil")
+    Oq = (dequant_mxfp8(eq["codes"], eq["sf"]) @ Vd) / E.sum(axis=1, keepdims=True)
+    return O, T_err, Oq, vmax
 
 
-def within_att_tol(O_test, O_ref, T_err) -> np.ndarray:
-    """Element-wise pass mask |O_test - O_ref| <= ATT_RTOL * T + ATT_ATOL."""
+def within_att_tol(O_test, O_ref, T_err, vmax) -> np.ndarray:
+    """Worst-case mask against the exact result:
+    |O_test - O_ref| <= ATT_RTOL * T + 2^-12 * vmax + ATT_ATOL."""
     O_test = np.asarray(O_test, dtype=np.float64)
-    return np.abs(O_test - np.asarray(O_ref, dtype=np.float64)) <= ATT_RTOL * np.asarray(T_err) + ATT_ATOL
+    bound = ATT_RTOL * np.asarray(T_err) + 2.0 ** -12 * np.asarray(vmax)[None, :] + ATT_ATOL
+    return np.abs(O_test - np.asarray(O_ref, dtype=np.float64)) <= bound
+
+
+def within_att_tight(O_test, O_q, T_err) -> np.ndarray:
+    """Mask against the oracle's own rounding of the weights:
+    |O_test - O_q| <= 2e-3 * T + 1e-6 (the GEMM's rule)."""
+    O_test = np.asarray(O_test, dtype=np.float64)
+    return np.abs(O_test - np.asarray(O_q, dtype=np.float64)) <= 2e-3 * np.asarray(T_err) + 1e-6

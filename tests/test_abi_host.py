@@ -280,3 +280,26 @@ def test_rceil_flag_and_scale_rule_checks():
     if not torch.cuda.is_available():
         assert _st(mxq.quantize_mxfp8, dev(SMALL), dev(SMALL), dev(SMALL), 4, 128, 128, None,
                    mxq.SCALE_RCEIL) == mxq.ERR_ARCH
+
+
+def test_attention_arguments_are_checked_on_the_host():
+    H, T, d = 2, 256, 128
+    need = mxq.attention_workspace_bytes(H, T, d)
+    assert need >= 3 * H * T * d and need % 256 == 0
+    assert mxq.attention_workspace_bytes(H, T, 64) == 0 and mxq.attention_workspace_bytes(0, T, d) == 0
+    q, k, v, o = (dev(H * T * d * 2) for _ in range(4))
+    ws = dev(need)
+
+    def call(H_=H, T_=T, d_=d, ws_=ws, nbytes=need, q_=q):
+        return mxq._attention_mxfp8(q_, k, v, H_, T_, d_, 0.0, o, ws_, nbytes, None)
+
+    assert call(d_=64) == mxq.ERR_UNSUPPORTED_SHAPE
+    assert call(T_=200) == mxq.ERR_UNSUPPORTED_SHAPE       # tokens % 128
+    assert call(H_=-1) == mxq.ERR_INVALID_ARG
+    assert call(nbytes=need - 1) == mxq.ERR_WORKSPACE
+    assert call(ws_=ws + 16) == mxq.ERR_ALIGNMENT
+    assert call(q_=q + 2) == mxq.ERR_ALIGNMENT
+    assert call(q_=None) == mxq.ERR_INVALID_ARG
+    assert call(H_=0) == mxq.OK                              # nothing to do
+    if not torch.cuda.is_available():
+        assert call() == mxq.ERR_ARCH                        # past every argument check

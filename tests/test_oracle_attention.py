@@ -5,7 +5,8 @@ softmax or matmul), softmax invariants, closed forms (equal keys give the
 mean of the values, equal values pass through, two keys give the logistic
 function), inputs that MXFP8 represents exactly (the quantised attention
 must then equal the plain one), and the derived error bound (it holds for
-the quantisation of P, and it rejects a planted scale mistake).
+the rounding of the weights, and the sharp check rejects a planted scale
+mistake and a dropped key block).
 """
 
 import math
@@ -69,11 +70,11 @@ def test_exactly_representable_inputs_give_the_plain_attention():
     rng = np.random.default_rng(4)
     T, d = 64, 64
     Q, K, V = (_exact_mx(rng, T, d) for _ in range(3))
-    O, Terr, Oq = A.attention_ref(_bf16(Q), _bf16(K), _bf16(V))
+    O, Terr, Oq, vmax = A.attention_ref(_bf16(Q), _bf16(K), _bf16(V))
     assert np.allclose(O, A.attention_plain(Q, K, V), rtol=0, atol=1e-13)
     assert np.all(Terr + 1e-15 >= np.abs(O))
-    # the P rounding moves the result by less than the derived bound
-    assert A.within_att_tol(Oq, O, Terr).all()
+    # the rounding of the weights moves the result by less than the derived bound
+    assert A.within_att_tol(Oq, O, Terr, vmax).all()
 
 
 def test_equal_keys_average_the_values():
@@ -82,7 +83,7 @@ def test_equal_keys_average_the_values():
     Q = _exact_mx(rng, T, d)
     K = np.tile(_exact_mx(rng, 1, d), (T, 1))
     V = _exact_mx(rng, T, d)
-    O, _, _ = A.attention_ref(_bf16(Q), _bf16(K), _bf16(V))
+    O, _, _, _ = A.attention_ref(_bf16(Q), _bf16(K), _bf16(V))
     assert np.allclose(O, np.tile(V.astype(np.float64).mean(axis=0), (T, 1)), atol=1e-14)
 
 
@@ -92,7 +93,7 @@ def test_equal_values_pass_through():
     Q, K = (rng.normal(size=(T, d)).astype(np.float32) for _ in range(2))
     v = np.float32(2.0 ** -3) * rng.integers(1, 8, size=d).astype(np.float32)
     V = np.tile(v, (T, 1))
-    O, _, _ = A.attention_ref(_bf16(Q), _bf16(K), _bf16(V))
+    O, _, _, _ = A.attention_ref(_bf16(Q), _bf16(K), _bf16(V))
     assert np.allclose(O, np.tile(v.astype(np.float64), (T, 1)), atol=1e-14)
 
 
@@ -108,17 +109,24 @@ def test_two_key_closed_form():
     assert np.allclose(A.attention_plain(Q, K, V)[0], want, atol=1e-14)
 
 
-def test_bound_holds_for_p_rounding_and_rejects_a_scale_mistake():
-    rng = np.random.default_rng(7)
+def test_bounds_hold_for_the_weight_rounding_and_reject_planted_mistakes():
     T, d = 256, 128
     Q, K, V = (torch.randn(T, d, generator=torch.Generator().manual_seed(s)).bfloat16() for s in (1, 2, 3))
-    O, Terr, Oq = A.attention_ref(Q, K, V)
-    assert A.within_att_tol(Oq, O, Terr).all()
-    # a kernel that forgot the 1/sqrt(d) softmax scale fails the bound
-    Obad, _, _ = A.attention_ref(Q, K, V, tau=1.0)
-    assert not A.within_att_tol(Obad, O, Terr).all()
+    O, Terr, Oq, vmax = A.attention_ref(Q, K, V)
+    assert A.within_att_tol(Oq, O, Terr, vmax).all()
+    assert np.all(Terr + 1e-15 >= np.abs(O))
+    # a kernel that forgot the 1/sqrt(d) softmax scale fails both checks
+    Obad, _, _, _ = A.attention_ref(Q, K, V, tau=1.0)
+    assert not A.within_att_tol(Obad, O, Terr, vmax).all()
+    assert A.within_att_tight(Obad, Oq, Terr).mean() < 0.5
+    # so does one that left the weights unrounded ... only for a few elements:
+    # the sharp check separates O from O_q on most of them
+    assert A.within_att_tight(O, Oq, Terr).mean() < 0.9
+    # a kernel that dropped the last key block fails the sharp check
+    Od, _, _, _ = A.attention_ref(Q[:, :], K[: T - 32], V[: T - 32])
+    assert A.within_att_tight(Od, Oq, Terr).mean() < 0.5
     # rows restrict the queries only
     rows = np.array([0, 5, 255])
-    O2, T2, _ = A.attention_ref(Q, K, V, rows=rows)
+    O2, T2, Oq2, v2 = A.attention_ref(Q, K, V, rows=rows)
     assert np.allclose(O2, O[rows], atol=1e-15) and np.allclose(T2, Terr[rows], atol=1e-15)
-    del rng
+    assert np.allclose(Oq2, Oq[rows], atol=1e-15) and np.array_equal(v2, vmax)

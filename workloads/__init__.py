@@ -31,6 +31,7 @@ __all__ = [
     "make_case",
     "random_case",
     "flux_linear_stack",
+    "flux_attention",
     "CONFIG_NAMES",
 ]
 
@@ -200,3 +201,17 @@ def flux_linear_stack(batch: int = 1, n_double: int = 19, n_single: int = 38,
             dict(name=f"s{b}.linear2", M=Ms, K=hidden + mlp, N=hidden),
         ]
     return layers
+
+
+def flux_attention(heads: int = 24, tokens: int = 4608, d: int = 128, seed: int = 0):
+    """Q, K, V [heads, tokens, d] bf16 of one FLUX-shaped attention (24 heads of
+    128 channels over 4096 image + 512 text tokens at 1024 x 1024).
+
+    Draw order: Q, K, V ~ N(0, 1) (the queries and keys of a FLUX block are
+    RMS-normalised, so unit-scale entries are the plain stand-in).
+    """
+    g = _gen(seed)
+    Q = torch.randn(heads, tokens, d, generator=g)
+    K = torch.randn(heads, tokens, d, generator=g)
+    V = torch.randn(heads, tokens, d, generator=g)
+    return Q.bfloat16(), K.bfloat16(), V.bfloat16()
