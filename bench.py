@@ -1,6 +1,6 @@
 """Benchmark of the microscaled linear layer on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3|c2|c4|c1|c5]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3|c2|c4|c1|c5|attn|bf16]
                     [--batch 1|4] [--impl mxq|reference] [--shape M,K,N --fmt nvfp4|mxfp8]
 
 A step is one pass of the whole hot path over one batch of synthetic input:
@@ -17,12 +17,15 @@ ranks.  The GEMM's own duration (the roofline's kernel) comes from an event
 pair that mxq_linear records around its GEMM launch in every timed step.  Each step uses one of several rotating buffer sets whose total size
 is well above the 126 MB L2, so no step starts with its inputs in L2.  Under
 torchrun each rank runs an independent replica (weak scaling: no data-path
-collective; the path does not shard).
+collective between replicas).
 
 --workload c5 times a whole FLUX-shaped linear stack instead (about 300
 layers per pass, mixed NVFP4 / bf16 by the selective rule; eager and replayed
 from a CUDA graph) against the same stack in bf16 through cuBLAS; use a small
---steps there (one pass is ~17 ms at batch 1).
+--steps there (one pass is ~17 ms at batch 1).  --workload attn times the
+8-bit attention (24 heads x 4608 tokens x 128) against bf16 SDPA;
+--workload bf16 times the dispatcher's bf16 branch against torch.addmm on
+the stack's bf16 layers.
 
 --impl reference times the CPU oracle (the plain numpy restatement of the
 method) on a bounded sample of the same workload on the host cores.
@@ -63,7 +66,7 @@ NOMINAL_RATIO = {"nvfp4": 4.0, "mxfp8": 2.0, "bf16": 1.0}
 # DRAM bytes (read + write) of one launch of the roofline's kernel, from one
 # ncu capture of the committed kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum); None where no capture of the current kernel exists.
-GEMM_TRAFFIC_BYTES = {}
+GEMM_TRAFFIC_BYTES = {"c3_nvfp4_4608x3072x12288": 92455680}
 
 
 def _peaks():
@@ -657,14 +660,125 @@ def run_stack(args, rank, world, local_rank):
     }
 
 
+def run_bf16_branch(args, rank, world, local_rank):
+    """The dispatcher's bf16 branch against cuBLAS.  Every distinct layer
+    shape of the FLUX-shaped stack that the selective rule keeps in bf16
+    (batch 1: the modulation layers at M = 1 and the text stream's layers at
+    M = 512; batch 4: the modulation layers at M = 4) runs through
+    mxq_linear (the library's own tcgen05 bf16 GEMM) and through torch.addmm
+    on the same bf16 weights, bias and buffers.  Weight sets rotate so that
+    more than 2 x L2 of weights stream between two uses of one set.  The
+    line's value is the stack's bf16-layer flops over the summed per-layer
+    time of the library, each shape weighted by its count in the stack."""
+    import fp8_gemm_diffusion_b200 as mxq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    counts = {}
+    for l in workloads.flux_linear_stack(batch=args.batch):
+        key = (l["M"], l["K"], l["N"])
+        counts[key] = counts.get(key, 0) + 1
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    rows, launches = [], 0
+    tot_flops = tot_mxq = tot_ref = 0.0
+    probe = None
+    for (M, K, N), cnt in counts.items():
+        W0 = (torch.randn(N, K, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        b0 = (torch.randn(N, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        w0 = mxq.Weight(W0, b0, fmt="nvfp4")
+        if mxq.linear_path(w0.handle, M) != mxq.BF16:
+            continue
+        nsets = max(2, -(-(256 << 20) // (N * K * 2)))
+        sets = [(W0, b0, w0)] + [
+            ((W := (torch.randn(N, K, generator=g, device=dev) * 0.02).to(torch.bfloat16)),
+             (b := (torch.randn(N, generator=g, device=dev) * 0.02).to(torch.bfloat16)),
+             mxq.Weight(W, b, fmt="nvfp4")) for _ in range(nsets - 1)]
+        x = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        y_ref = torch.empty_like(y)
+        ws_bytes = max(256, mxq.linear_workspace_bytes(M, K, mxq.BF16))
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+        def ours(i, sets=sets, x=x, y=y, ws=ws, ws_bytes=ws_bytes, M=M):
+            mxq.linear(sets[i % len(sets)][2].handle, x, M, y, ws, ws_bytes, stream=stream)
+
+        def cublas(i, sets=sets, x=x, y_ref=y_ref):
+            W, b, _ = sets[i % len(sets)]
+            torch.addmm(b, x, W.t(), out=y_ref)
+
+        def timed(fn, n):
+            for i in range(args.warmup):
+                fn(i)
+            torch.cuda.synchronize()
+            torch.cuda._sleep(SPIN_CYCLES)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(n):
+                fn(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return max_over_ranks(e0.elapsed_time(e1), dev) / n
+
+        n = max(args.steps, 3 * nsets)
+        ms_ours = timed(ours, n)
+        ms_ref = timed(cublas, n)
+        launches += n
+        if mxq.get_device_error() != mxq.OK:
+            raise RuntimeError("device-side timeout in the bf16 branch")
+        ours(0)
+        cublas(0)
+        torch.cuda.synchronize()
+        diff = (y.float() - y_ref.float()).abs().max().item()
+        flops = 2.0 * M * N * K
+        tot_flops += cnt * flops
+        tot_mxq += cnt * ms_ours
+        tot_ref += cnt * ms_ref
+        rows.append({"M": M, "K": K, "N": N, "count_in_stack": cnt, "us_mxq": round(ms_ours * 1e3, 2),
+                     "us_addmm": round(ms_ref * 1e3, 2), "addmm_over_mxq": round(ms_ref / ms_ours, 3),
+                     "tflops_mxq": round(flops / (ms_ours * 1e-3) / 1e12, 1),
+                     "weight_gbs_mxq": round(N * K * 2 / (ms_ours * 1e-3) / 1e9, 1),
+                     "max_abs_diff_vs_addmm": diff})
+    value = tot_flops / (tot_mxq * 1e-3) / 1e12
+    peaks = _peaks()
+    return {
+        "metric": "bf16-branch GEMM TFLOPS over the FLUX stack's bf16 layers (stack-weighted)",
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(tot_mxq, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 operands, fp32 accumulate, bf16 out",
+        "data": "synthetic (seeded FLUX-shaped layers; random-init weights)",
+        "config": {"workload": f"c5_bf16_layers_b{args.batch}", "parallelism": f"replicas x{world}",
+                   "step": "each bf16-path layer of the stack once, through mxq_linear",
+                   "l2": "rotating weight sets, > 256 MiB of weights between two uses of a set"},
+        "per_shape": rows,
+        "bf16_baseline": {"impl": "torch.addmm bf16 (cuBLAS), same weights and buffers",
+                          "value": round(tot_flops / (tot_ref * 1e-3) / 1e12, 2), "unit": UNIT,
+                          "ms_per_step": round(tot_ref, 5), "speedup_of_value": round(tot_ref / tot_mxq, 3)},
+        "roofline": {"kernel": "gemm_kernel<BF16> / gemm_pair_kernel<BF16>", "bound": "hbm",
+                     "note": "the M = 1 and M = 512 layers stream their weights; see per_shape weight_gbs_mxq",
+                     "peak": peaks["hbm"], "unit": "GB/s", "achieved": None, "frac": None, "traffic": None},
+        "e2e": None,
+        "gpu_launches": launches,
+        "cpu_baseline": None,
+    }
+
+
 # ------------------------------------------------------------- attention
 def run_attention(args, rank, world, local_rank):
     """One step = one FLUX-shaped attention (24 heads x 4608 tokens x 128)
     through mxq_attention_mxfp8: per-token MXFP8 of Q and K, MXFP8 of V^T,
-    then the attention kernel.  The metric counts the attention's two
-    products, 4 * heads * tokens^2 * d per step (the kernel runs the first
-    product twice, once per softmax pass: 6 * heads * tokens^2 * d on the
-    tensor cores, which the roofline uses).  Baseline: PyTorch's
+    then the attention kernel (one pass over the keys).  The metric counts
+    the attention's two products, 4 * heads * tokens^2 * d per step, which
+    is also what the tensor cores run.  Baseline: PyTorch's
     scaled_dot_product_attention in bf16 on the same tensors."""
     import torch.nn.functional as Fn
 
@@ -680,7 +794,7 @@ def run_attention(args, rank, world, local_rank):
     nbytes = mxq.attention_workspace_bytes(H, T, d)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     flops = 4.0 * H * T * T * d
-    mma_flops = 6.0 * H * T * T * d
+    mma_flops = flops
 
     def step(i):
         q, k, v, o = sets[i % nsets]
@@ -750,7 +864,7 @@ def run_attention(args, rank, world, local_rank):
         "data": "synthetic (seeded FLUX-shaped Q, K, V ~ N(0, 1))",
         "config": {"workload": f"flux_attention_{H}x{T}x{d}", "heads": H, "tokens": T, "head_dim": d,
                    "parallelism": f"replicas x{world}",
-                   "step": "mxq_attention_mxfp8: MXFP8 of Q, K (per token) and V^T, two-pass softmax attention",
+                   "step": "mxq_attention_mxfp8: MXFP8 of Q, K (per token) and V^T, one-pass softmax attention",
                    "l2": f"rotating {nsets} input sets ({nsets * 4 * H * T * d * 2 / 2**20:.0f} MiB > 126 MiB L2)"},
         "kernels_ms": {"step": round(step_ms, 5), "call_with_events": round(call_ms, 5)},
         "roofline": {"kernel": "attention_mxfp8_kernel + quantisers", "bound": "tensor",
@@ -758,7 +872,7 @@ def run_attention(args, rank, world, local_rank):
                      "unit": "TFLOP/s", "frac": round(mma_flops / (step_ms * 1e-3) / 1e12 / peak, 4),
                      "peak_kind": "burst",
                      "peak_source": f"{peaks['source']} bf16 burst x 2 (nominal fp8:bf16 dense ratio); "
-                                    "achieved counts the 6 H T^2 d tensor-core flops the kernel runs",
+                                    "achieved counts the 4 H T^2 d tensor-core flops of the step",
                      "traffic": None},
         "bf16_baseline": {"impl": "torch scaled_dot_product_attention, bf16, same tensors",
                           "value": round(whole_job_tflops(world, 1, flops, bf16_ms), 2), "unit": UNIT,
@@ -825,7 +939,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5", "attn"])
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5", "attn", "bf16"])
     ap.add_argument("--batch", type=int, default=1, choices=[1, 4],
                     help="batch of the c5 stack (1: 4608 tokens per image)")
     ap.add_argument("--impl", default="mxq", choices=["mxq", "reference"])
@@ -848,7 +962,7 @@ def main():
         # the CPU oracle on the host cores: rank 0 only, a few bounded samples
         if rank != 0:
             return 0
-        if args.workload in ("c5", "attn"):
+        if args.workload in ("c5", "attn", "bf16"):
             print(json.dumps({"impl": "reference", "unavailable": "the oracle arm times single "
                               "linear layers (c1-c4)"}))
             return 0
@@ -880,8 +994,9 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device("cuda", local_rank))
     try:
-        if args.workload in ("c5", "attn"):
-            result = (run_stack if args.workload == "c5" else run_attention)(args, rank, world, local_rank)
+        if args.workload in ("c5", "attn", "bf16"):
+            fn = {"c5": run_stack, "attn": run_attention, "bf16": run_bf16_branch}[args.workload]
+            result = fn(args, rank, world, local_rank)
             if rank == 0:
                 print(json.dumps(result))
             return 0

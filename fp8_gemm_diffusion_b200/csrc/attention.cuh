@@ -9,27 +9,41 @@
 //   Qq = MXFP8(Q), Kq = MXFP8(K)       scales per token and per 32 channels
 //   Vq = MXFP8(V^T)                    scales per channel and per 32 tokens
 //   S  = deq(Qq) deq(Kq)^T             block-scaled MMAs, fp32 in tensor memory
-//   m  = rowmax(S)                     first pass over the key blocks
-//   E  = 2^((S - m) * tau * log2 e)    second pass, fp32, in [0, 1]
+//   t  = S * tau * log2 e
+//   E  = 2^(t - m), m an integer       fp32
 //   Eq = MXFP8(E) along keys, ceiling scale rule (no saturation)
-//   O  = deq(Eq) deq(Vq)^T / rowsum(E) block-scaled MMAs, fp32; bf16 out
+//   O  = deq(Eq) deq(Vq)^T / rowsum(deq(Eq))   block-scaled MMAs, fp32; bf16 out
 //
-// Two passes over the keys keep the softmax exact without rescaling the
-// output accumulator: the first finds each row's maximum (no exponentials),
-// the second weights every key against the final maximum.
+// One pass over the keys.  Softmax is the same for every m; with m an
+// integer the MXFP8 codes are the same for every m too (2^k times a block
+// moves its shared exponent by k and leaves the codes), so m can be a
+// running maximum: the first key block sets m = ceil(max t), and a later
+// block whose maximum exceeds m by more than 8 raises it, after the output
+// accumulator and the row sum are multiplied by 2^(m_old - m_new), exactly.
+// Weights up to 2^8 stay far inside fp32, and the result is the one the
+// final maximum would have given.  The row sums of the quantised weights
+// come out of the second product: V^T carries 16 extra rows (a row of ones,
+// then zeros) with unit scales, so O has a 129th column = sum_j deq(Eq)_j,
+// rescaled with O and divided out at the end.
 //
-// One CTA per (head, 128-query tile), 6 warps:
+// One CTA per (head, 128-query tile), 12 warps:
 //   warp 0      TMA producer: the Q tile and its scales once, then a ring of
-//               K blocks (first pass) and K + V^T blocks (second pass), each
-//               with its 512-byte scale chunks;
+//               key blocks (K, V^T and their 512-byte scale chunks);
 //   warp 1      tensor memory; one lane issues the scale copies (tcgen05.cp)
-//               and the MMAs: S = Q K^T into one of two S buffers, and
-//               O += Eq V^T behind the softmax of the same block;
-//   warps 2-5   softmax, one query row per thread (tensor-memory sub-partition
-//               warp % 4): row maxima, then weights, row sums, MXFP8 codes of
-//               E into shared memory (the MMA's A operand) and their scales
-//               into tensor memory; at the end O / rowsum -> bf16.
-// Every wait is bounded (ptx.cuh).
+//               and the MMAs: S = Q K^T of block j into S buffer j % 2, and
+//               O += Eq V^T of block j once its weights are in place;
+//   warps 4-7   softmax of the even key blocks, warps 8-11 of the odd ones
+//               (tensor-memory sub-partition warp % 4, one query row per
+//               thread): the two warpgroups work on consecutive blocks at
+//               the same time, each hiding the other's waits.  Per block:
+//               block maxima, the normaliser (taken over from the other
+//               warpgroup's previous block through shared memory and raised
+//               if needed), weights, MXFP8 codes of E into shared memory
+//               (the second product's A operand) and their scales into
+//               tensor memory; at the end O / rowsum -> bf16.
+// Every wait is bounded (ptx.cuh).  The softmax warps never leave their
+// loop early: after a timeout they skip the work but keep the hand-over
+// order, so no warp waits on a named barrier that is never signalled.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -45,22 +59,41 @@ namespace mxq {
 constexpr int kAttD = 128;       // head dimension
 constexpr int kAttTile = 128;    // query rows per CTA = keys per block
 constexpr int kAttStages = 4;
+constexpr float kAttRescale = 8.0f;  // raise m when a block's maximum exceeds it by more
 
 struct AttCfg {
   static constexpr int TILE_BYTES = kAttTile * 128;                 // 128 rows x 128 bytes (E4M3)
-  static constexpr int STAGE_BYTES = 2 * TILE_BYTES + 1024;         // K, V^T, their scale chunks
+  static constexpr int EXT_BYTES = 16 * 128;                        // V^T rows 128..143: ones, then zeros
+  // a stage: K, V^T and its 16-row extension (one B operand of 144 rows), K scales, V^T scales
+  static constexpr int ST_EXT = 2 * TILE_BYTES, ST_KSF = ST_EXT + EXT_BYTES, ST_VSF = ST_KSF + 512;
+  static constexpr int STAGE_BYTES = ST_VSF + 512;                  // 35 KB (multiple of 1024)
   static constexpr int OFF_QSF = TILE_BYTES;                        // Q scale chunk (512 B)
+  static constexpr int OFF_ONESF = TILE_BYTES + 512;                // unit scales of the extension rows
   static constexpr int OFF_STAGE = TILE_BYTES + 1024;
   static constexpr int OFF_P = OFF_STAGE + kAttStages * STAGE_BYTES;  // two E-code buffers
-  static constexpr int OFF_BAR = OFF_P + 2 * TILE_BYTES;
+  static constexpr int OFF_XCH = OFF_P + 2 * TILE_BYTES;            // [128 rows] normaliser, [4] flags
+  static constexpr int XCH_BYTES = 128 * 4 + 64;
+  static constexpr int OFF_BAR = OFF_XCH + XCH_BYTES;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + OFF_BAR + BAR_BYTES;
-  // tensor memory columns: two S buffers, O, then scale sets of 4 columns
-  static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 384, T_KSF = 388, T_VSF = 392, T_PSF = 396;
+  // the second product has N = 144: d = 128 output columns, column 128 the
+  // row sum of the quantised weights (times the extension's row of ones),
+  // 15 zero columns
+  static constexpr int PV_N = kAttD + 16;
+  // tensor memory columns: two S buffers, O (144), scale columns of Q, K,
+  // V^T (two 128-row groups: the tile's and the extension's), and of the
+  // weights (one 4-column group per S buffer)
+  static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 400, T_KSF = 404, T_VSF = 408, T_PSF = 416;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int THREADS = 192;
-  static constexpr int SOFT_WARP0 = 2;
+  static constexpr int THREADS = 384;
+  static constexpr int SOFT_WARP0 = 4;
+  // registers: launched with 65536 / 384 = 168 per thread; the control
+  // warpgroup gives up registers so that a softmax thread holds its row of S
+  static constexpr int REGS_CTRL = 56, REGS_SOFT = 224;
 };
+static_assert(AttCfg::STAGE_BYTES % 1024 == 0, "stage alignment (128-byte swizzle atoms)");
+static_assert(AttCfg::T_PSF + 8 <= AttCfg::TMEM_COLS && AttCfg::T_O + AttCfg::PV_N <= AttCfg::T_QSF, "tensor memory");
+static_assert(128 * AttCfg::REGS_CTRL + 256 * AttCfg::REGS_SOFT <= 384 * 168, "register split");
 
 struct AttArgs {
   int heads, tokens;
@@ -77,14 +110,36 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// MXFP8 shared exponent by the ceiling rule: the smallest X with
-// bmax <= 448 * 2^X (bmax > 0), clamped to [-127, 127].
-__device__ __forceinline__ int mx_ceil_exponent(float bmax) {
-  if (!(bmax > 0.0f)) return -127;
-  const int e = floor_log2_f32(bmax);
-  int X = e - 8;
-  if (static_cast<double>(bmax) > ldexp(1.75, e)) X += 1;  // bmax > 448 * 2^(e - 8)
+// MXFP8 shared exponent by the ceiling rule for a block maximum that is 0
+// or a normal fp32: the smallest X with bmax <= 448 * 2^X, clamped to
+// [-127, 127].  With bmax = (1 + f) 2^e, 448 * 2^(e - 8) = 1.75 * 2^e, so X is
+// e - 8, plus one when the fraction f exceeds 0.75 (bits above 0x600000).
+__device__ __forceinline__ int mx_ceil_exponent_normal(float bmax) {
+  const uint32_t b = __float_as_uint(bmax);
+  if (b == 0u) return -127;
+  const int X = static_cast<int>(b >> 23) - 127 - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
   return min(max(X, -127), 127);
+}
+
+// Instruction descriptor of an M = 128 kind::mxf8f6f4 MMA (E4M3 x E4M3,
+// UE8M0 scales) with separate scale-byte selectors for A and B.
+__device__ __forceinline__ uint32_t idesc_mxfp8_m128(int n, uint32_t a_id, uint32_t b_id) {
+  return (b_id << 4) | ((static_cast<uint32_t>(n) >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24) | (a_id << 29);
+}
+
+__device__ __forceinline__ float max32(const uint32_t* u) {
+  float a = fmaxf(__uint_as_float(u[0]), __uint_as_float(u[1]));
+  float b = fmaxf(__uint_as_float(u[2]), __uint_as_float(u[3]));
+  float c = fmaxf(__uint_as_float(u[4]), __uint_as_float(u[5]));
+  float d = fmaxf(__uint_as_float(u[6]), __uint_as_float(u[7]));
+#pragma unroll
+  for (int i = 8; i < 32; i += 4) {
+    a = fmaxf(a, __uint_as_float(u[i]));
+    b = fmaxf(b, __uint_as_float(u[i + 1]));
+    c = fmaxf(c, __uint_as_float(u[i + 2]));
+    d = fmaxf(d, __uint_as_float(u[i + 3]));
+  }
+  return fmaxf(fmaxf(a, b), fmaxf(c, d));
 }
 
 __global__ void __launch_bounds__(AttCfg::THREADS, 1)
@@ -108,6 +163,7 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
   const uint32_t o_full = bar + 8u + 8u * (2 * kAttStages + 8);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_BAR + 8 * (2 * kAttStages + 10));
   static_assert(8 * (2 * kAttStages + 10) + 4 <= C::BAR_BYTES, "barrier area");
+  constexpr int NSOFT = 4;  // warps of one softmax warpgroup (the one that owns S / P buffer b)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = args.tokens;
@@ -123,8 +179,8 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full(b), 1);
-      mbar_init(s_free(b), 4);
-      mbar_init(p_full(b), 4);
+      mbar_init(s_free(b), NSOFT);
+      mbar_init(p_full(b), NSOFT);
       mbar_init(p_free(b), 1);
     }
     mbar_init(o_full, 1);
@@ -137,6 +193,18 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
+  // constant operand bytes, read by the MMAs through the async proxy: each
+  // stage's V^T extension (row 128 = E4M3 1.0 = 0x38 in every key, rows
+  // 129..143 zero; a row of equal bytes needs no swizzle) and a 512-byte
+  // chunk of unit scales (E8M0 127)
+  for (int i = threadIdx.x; i < kAttStages * C::EXT_BYTES / 16; i += C::THREADS) {
+    const int st = i / (C::EXT_BYTES / 16), o = i % (C::EXT_BYTES / 16);
+    const uint32_t v = o < 8 ? 0x38383838u : 0u;
+    *reinterpret_cast<uint4*>(base_ptr + C::OFF_STAGE + st * C::STAGE_BYTES + C::ST_EXT + 16 * o) = make_uint4(v, v, v, v);
+  }
+  for (int i = threadIdx.x; i < 512 / 16; i += C::THREADS)
+    *reinterpret_cast<uint4*>(base_ptr + C::OFF_ONESF + 16 * i) = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -144,6 +212,8 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
   grid_dep_wait();  // Q, K, V^T and their scales come from the quantisers just before
   grid_dep_launch();
 
+  if (warp < C::SOFT_WARP0) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_CTRL));
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -153,20 +223,16 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
       int s = 0, issued = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int g = 0; g < 2 * nkb; ++g) {
-        const bool pv = g >= nkb;
-        const int kb = pv ? g - nkb : g;
+      for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait_bounded(kv_empty(s), ph ^ 1u)) { ok = false; break; }
         const uint32_t st = base + C::OFF_STAGE + s * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(kv_full(s), (C::TILE_BYTES + 512) * (pv ? 2u : 1u));
+        mbar_arrive_expect_tx(kv_full(s), 2u * (C::TILE_BYTES + 512));
         const int krow = h * T + kb * kAttTile;
         tma_load_2d(st, &tmap_k, kv_full(s), 0, krow);
-        bulk_load(st + 2 * C::TILE_BYTES, args.k_sf + static_cast<int64_t>(krow / 128) * 512, 512, kv_full(s));
-        if (pv) {
-          tma_load_2d(st + C::TILE_BYTES, &tmap_v, kv_full(s), kb * kAttTile, h * kAttD);
-          bulk_load(st + 2 * C::TILE_BYTES + 512, args.v_sf + (static_cast<int64_t>(h) * nkb + kb) * 512, 512,
-                    kv_full(s));
-        }
+        bulk_load(st + C::ST_KSF, args.k_sf + static_cast<int64_t>(krow / 128) * 512, 512, kv_full(s));
+        tma_load_2d(st + C::TILE_BYTES, &tmap_v, kv_full(s), kb * kAttTile, h * kAttD);
+        bulk_load(st + C::ST_VSF, args.v_sf + (static_cast<int64_t>(h) * nkb + kb) * 512, 512,
+                  kv_full(s));
         ++issued;
         if (++s == kAttStages) { s = 0; ph ^= 1u; }
       }
@@ -184,157 +250,225 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
     if (lane == 0) {
       bool ok = mbar_wait_bounded(q_full, 0);
       tc_fence_after();
-      if (ok) tc_cp_32x128b_warpx4(tmem + C::T_QSF, desc_sf_chunk(base + C::OFF_QSF));
+      if (ok) {
+        tc_cp_32x128b_warpx4(tmem + C::T_QSF, desc_sf_chunk(base + C::OFF_QSF));
+        // unit scales of the V^T extension rows (128-row group 1 of the B scales), once
+        tc_cp_32x128b_warpx4(tmem + C::T_VSF + 4, desc_sf_chunk(base + C::OFF_ONESF));
+      }
       const uint64_t qdesc = desc_kmajor_sw128(base);
-      int s = 0, s_prev = 0;
-      uint32_t ph = 0;
-      // S[b] = Q K^T of the block in stage s (its scale chunk copied first;
-      // the copy follows the previous block's MMAs in this thread's order)
-      auto qk = [&](int g, int st_idx) {
-        const uint32_t st = base + C::OFF_STAGE + st_idx * C::STAGE_BYTES;
-        const int b = g & 1;
-        tc_cp_32x128b_warpx4(tmem + C::T_KSF, desc_sf_chunk(st + 2 * C::TILE_BYTES));
+      // S[j % 2] = Q K^T of key block j (stage j % kAttStages); its scale
+      // chunk is copied first, behind the previous MMAs in this thread's order
+      auto issue_qk = [&](int j) {
+        tc_fence_after();
+        const uint32_t st = base + C::OFF_STAGE + (j % kAttStages) * C::STAGE_BYTES;
+        tc_cp_32x128b_warpx4(tmem + C::T_KSF, desc_sf_chunk(st + C::ST_KSF));
         const uint64_t kdesc = desc_kmajor_sw128(st);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint64_t koff = static_cast<uint64_t>(2 * j);  // 32 bytes of d per MMA
-          mma_mxfp8(tmem + C::T_S + b * kAttTile, qdesc + koff, kdesc + koff, make_idesc<Fmt::MXFP8>(kAttTile, j),
-                    (tmem + C::T_QSF) | (static_cast<uint32_t>(j) << 30),
-                    (tmem + C::T_KSF) | (static_cast<uint32_t>(j) << 30), j > 0 ? 1u : 0u);
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t koff = static_cast<uint64_t>(2 * k);  // 32 bytes of d per MMA
+          mma_mxfp8(tmem + C::T_S + (j & 1) * kAttTile, qdesc + koff, kdesc + koff,
+                    idesc_mxfp8_m128(kAttTile, k, k), (tmem + C::T_QSF) | (static_cast<uint32_t>(k) << 30),
+                    (tmem + C::T_KSF) | (static_cast<uint32_t>(k) << 30), k > 0 ? 1u : 0u);
         }
-        tc_commit(s_full(b));
+        tc_commit(s_full(j & 1));
       };
-      // O += Eq V^T of key block kb (stage st_idx), once its weights are in place
-      auto pv_mma = [&](int kb, int st_idx) -> bool {
-        const int b = kb & 1;
-        if (!mbar_wait_bounded(p_full(b), (kb >> 1) & 1)) return false;
+      // O += Eq V^T of key block j; MMA k covers keys [32 k, 32 k + 32),
+      // scale byte k of the row's word
+      auto issue_pv = [&](int j) {
+        const int b = j & 1, st_idx = j % kAttStages;
         tc_fence_after();
         const uint32_t st = base + C::OFF_STAGE + st_idx * C::STAGE_BYTES;
-        tc_cp_32x128b_warpx4(tmem + C::T_VSF, desc_sf_chunk(st + 2 * C::TILE_BYTES + 512));
+        tc_cp_32x128b_warpx4(tmem + C::T_VSF, desc_sf_chunk(st + C::ST_VSF));
         const uint64_t pdesc = desc_kmajor_sw128(base + C::OFF_P + b * C::TILE_BYTES);
         const uint64_t vdesc = desc_kmajor_sw128(st + C::TILE_BYTES);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint64_t koff = static_cast<uint64_t>(2 * j);  // 32 keys per MMA
-          mma_mxfp8(tmem + C::T_O, pdesc + koff, vdesc + koff, make_idesc<Fmt::MXFP8>(kAttD, j),
-                    (tmem + C::T_PSF + 4 * b) | (static_cast<uint32_t>(j) << 30),
-                    (tmem + C::T_VSF) | (static_cast<uint32_t>(j) << 30), (kb > 0 || j > 0) ? 1u : 0u);
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t koff = static_cast<uint64_t>(2 * k);  // 32 keys per MMA
+          mma_mxfp8(tmem + C::T_O, pdesc + koff, vdesc + koff, idesc_mxfp8_m128(C::PV_N, k, k),
+                    (tmem + C::T_PSF + 4 * b) | (static_cast<uint32_t>(k) << 30),
+                    (tmem + C::T_VSF) | (static_cast<uint32_t>(k) << 30), (j > 0 || k > 0) ? 1u : 0u);
         }
         tc_commit(p_free(b));
         tc_commit(kv_empty(st_idx));
-        return true;
       };
-      for (int g = 0; g < 2 * nkb && ok; ++g) {
-        const bool pv = g >= nkb;
-        const int kb = pv ? g - nkb : g;
-        if (!mbar_wait_bounded(kv_full(s), ph)) { ok = false; break; }
-        // S buffer g & 1 was read by the softmax of block g - 2
-        if (!mbar_wait_bounded(s_free(g & 1), ((g >> 1) & 1) ^ 1u)) { ok = false; break; }
-        tc_fence_after();
-        qk(g, s);
-        if (!pv) {
-          tc_commit(kv_empty(s));  // first pass: K only
-        } else if (kb > 0) {
-          if (!(ok = pv_mma(kb - 1, s_prev))) break;
+      // Serve whichever is ready: S of block jq (its K has landed and the
+      // softmax has read S of block jq - 2 from the same buffer) or the
+      // product of block jp (its weights are in place).  The two warpgroups
+      // then run independently; the products stay in block order, which the
+      // rescaling of O relies on.  A stretch of 2 s without progress ends
+      // the loop with a timeout.
+      int jq = 0, jp = 0;
+      uint32_t idle = 0;
+      uint64_t t_idle = 0;
+      while (ok && jp < nkb) {
+        bool did = false;
+        if (jq < nkb && mbar_test(kv_full(jq % kAttStages), (jq / kAttStages) & 1) &&
+            mbar_test(s_free(jq & 1), ((jq >> 1) & 1) ^ 1u)) {
+          issue_qk(jq++);
+          did = true;
         }
-        s_prev = s;
-        if (++s == kAttStages) { s = 0; ph ^= 1u; }
+        if (jp < jq && mbar_test(p_full(jp & 1), (jp >> 1) & 1)) {
+          issue_pv(jp++);
+          did = true;
+        }
+        if (did) {
+          idle = 0;
+        } else if ((++idle & 255u) == 0u) {
+          const uint64_t now = globaltimer_ns();
+          if (idle == 256u) {
+            t_idle = now;
+          } else if (now - t_idle > kWaitLimitNs) {
+            record_error(kErrTimeout);
+            ok = false;
+          }
+        }
       }
-      if (ok) ok = pv_mma(nkb - 1, s_prev);
       tc_commit(o_full);
       // every MMA / copy issued above must finish before tensor memory is freed
       mbar_wait_bounded(o_full, 0);
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFT));
     // ------------------------------------------------------------ softmax
-    const int q = warp & 3;            // tensor-memory sub-partition
-    const int r = q * 32 + lane;       // query row of the tile
+    const int q = warp & 3;                        // tensor-memory sub-partition
+    const int G = (warp - C::SOFT_WARP0) >> 2;     // 0: even key blocks, 1: odd
+    const int r = q * 32 + lane;                   // query row of the tile
     const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    // named barriers of sub-partition q: normaliser hand-over even -> odd
+    // (2 + q) and odd -> even (6 + q), final row sums (10 + q); 64 threads
+    const uint32_t bar_to_other = (G == 0 ? 2u : 6u) + static_cast<uint32_t>(q);
+    const uint32_t bar_from_other = (G == 0 ? 6u : 2u) + static_cast<uint32_t>(q);
+    float* const xm = reinterpret_cast<float*>(base_ptr + C::OFF_XCH);               // [128] normaliser
+    volatile int* const xok = reinterpret_cast<volatile int*>(xm + 128);             // [4] sub-partition flags
     const float c = args.c;
-    uint32_t u[kAttTile];  // one row of S (fp32 bits), then of E, then of O
+    uint32_t u[kAttTile];  // the row of S (fp32 bits) of the current block, then of O
     bool ok = true;
-    float m = -INFINITY;
-    auto load_s = [&](int g) -> bool {
-      if (!mbar_wait_bounded(s_full(g & 1), (g >> 1) & 1)) return false;
-      tc_fence_after();
+    float m = -INFINITY;   // normaliser in effect (an integer once set)
+    for (int j = G; j < nkb; j += 2) {
+      const int b = j & 1;  // == G
+      const bool got = __all_sync(0xffffffffu, ok && mbar_wait_bounded(s_full(b), (j >> 1) & 1));
+      if (got) {
+        tc_fence_after();
 #pragma unroll
-      for (int i = 0; i < kAttTile / 32; ++i)
-        tmem_ld_32x32b_x32_nowait(trow + C::T_S + (g & 1) * kAttTile + 32 * i, u + 32 * i);
-      tc_wait_ld();
+        for (int i = 0; i < kAttTile / 32; ++i) tmem_ld_32x32b_x32_nowait(trow + C::T_S + b * kAttTile + 32 * i, u + 32 * i);
+        tc_wait_ld();
 #pragma unroll
-      for (int i = 0; i < kAttTile / 32; ++i) reg_fence32(u + 32 * i);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free(g & 1));  // S buffer read
-      return true;
-    };
-    // first pass: row maxima
-    for (int g = 0; g < nkb && ok; ++g) {
-      if (!(ok = load_s(g))) break;
-#pragma unroll
-      for (int i = 0; i < kAttTile; ++i) m = fmaxf(m, __uint_as_float(u[i]));
-    }
-    // second pass: weights against the final maximum, row sums, MXFP8 codes
-    const float mc = m * c;
-    float l = 0.0f;
-    for (int kb = 0; kb < nkb && ok; ++kb) {
-      if (!(ok = load_s(nkb + kb))) break;
-#pragma unroll
-      for (int i = 0; i < kAttTile; ++i) {
-        const float e = ex2_approx(fmaf(__uint_as_float(u[i]), c, -mc));
-        u[i] = __float_as_uint(e);
-        l += e;
+        for (int i = 0; i < kAttTile / 32; ++i) reg_fence32(u + 32 * i);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free(b));  // S buffer read
       }
+      ok = got;
+      float bm[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) bm[k] = max32(u + 32 * k);
+      const float tmax = fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3])) * c;
+      // the normaliser after block j - 1, from the other warpgroup
+      if (j >= 1) {
+        named_bar_sync(bar_from_other, 64);
+        m = xm[r];
+        ok = ok && xok[q] != 0;
+      }
+      const bool raise = tmax > m + kAttRescale;
+      const float m_new = raise ? ceilf(tmax) : m;
+      if (j + 1 < nkb) {
+        xm[r] = m_new;
+        __syncwarp();
+        if (lane == 0) xok[q] = ok ? 1 : 0;
+        named_bar_arrive(bar_to_other, 64);
+      }
+      // rows that raise the normaliser rescale O and its row-sum column by
+      // 2^(m - m_new) (the others by 1) once the product of block j - 1 is
+      // complete; the product of block j is issued only after this warp's
+      // p_full arrival below
+      if (j >= 1 && __any_sync(0xffffffffu, raise)) {
+        const int dm = raise ? static_cast<int>(m - m_new) : 0;  // <= -9 where raised
+        const float f = dm < -127 ? 0.0f : exp2_int(dm);
+        ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(p_free((j - 1) & 1), ((j - 1) >> 1) & 1));
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int g = 0; g < kAttD / 32; ++g) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32_nowait(trow + C::T_O + 32 * g, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            uint32_t w[16];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+              for (int k = 0; k < 16; ++k) w[k] = o[16 * h2 + k];
+              tmem_st_32x32b_x16(trow + C::T_O + 32 * g + 16 * h2, w);
+            }
+          }
+          uint32_t lsum = tmem_ld_32x32b_x1_nowait(trow + C::T_O + kAttD);
+          tc_wait_ld();
+          asm volatile("" : "+r"(lsum)::"memory");
+          tmem_st_32x32b_x1(trow + C::T_O + kAttD, __float_as_uint(__uint_as_float(lsum) * f));
+          tc_wait_st();
+        }
+      }
+      m = m_new;
+      // weights of the four 32-key blocks, their MXFP8 codes and scales (the
+      // row sum of the quantised weights comes out of the second product)
       uint32_t codes[kAttTile / 4];
       uint32_t sfw = 0;
 #pragma unroll
-      for (int blk = 0; blk < kAttTile / 32; ++blk) {
-        float bmax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) bmax = fmaxf(bmax, __uint_as_float(u[32 * blk + i]));
-        const int X = mx_ceil_exponent(bmax);
-        const float mult = exp2_int(-X);
+      for (int blk = 0; blk < 4; ++blk) {
+        const float emax = ex2_approx(fmaf(bm[blk], c, -m));
+        const int X = mx_ceil_exponent_normal(emax);
+        const float mx = m + static_cast<float>(X);  // E / 2^X = 2^(t - m - X)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int k0 = 32 * blk + 4 * i;
-          codes[8 * blk + i] = cvt_e4m3x2(__uint_as_float(u[k0]) * mult, __uint_as_float(u[k0 + 1]) * mult) |
-                               (cvt_e4m3x2(__uint_as_float(u[k0 + 2]) * mult, __uint_as_float(u[k0 + 3]) * mult) << 16);
+          const uint32_t* v = u + 32 * blk + 4 * i;
+          const float e0 = ex2_approx(fmaf(__uint_as_float(v[0]), c, -mx));
+          const float e1 = ex2_approx(fmaf(__uint_as_float(v[1]), c, -mx));
+          const float e2 = ex2_approx(fmaf(__uint_as_float(v[2]), c, -mx));
+          const float e3 = ex2_approx(fmaf(__uint_as_float(v[3]), c, -mx));
+          codes[8 * blk + i] = cvt_e4m3x2(e0, e1) | (cvt_e4m3x2(e2, e3) << 16);
         }
         sfw |= static_cast<uint32_t>(X + 127) << (8 * blk);
       }
-      const int b = kb & 1;
-      // the MMA of key block kb - 2 has read this buffer and its scales
-      if (!(ok = mbar_wait_bounded(p_free(b), ((kb >> 1) & 1) ^ 1u))) break;
-      tc_fence_after();
-      // row r of the A operand: 128 bytes, 128-byte swizzle (chunk c at c ^ (r % 8))
-      const uint32_t prow = base + C::OFF_P + b * C::TILE_BYTES + r * 128;
+      // the product of block j - 2 (this warpgroup's previous block) has read
+      // this buffer and its scales
+      ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(p_free(b), ((j >> 1) & 1) ^ 1u));
+      if (ok) {
+        tc_fence_after();
+        // row r of the A operand: 128 bytes, 128-byte swizzle (chunk ch at ch ^ (r % 8))
+        const uint32_t prow = base + C::OFF_P + b * C::TILE_BYTES + r * 128;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t addr = prow + ((ch ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(codes[4 * ch]),
-                     "r"(codes[4 * ch + 1]), "r"(codes[4 * ch + 2]), "r"(codes[4 * ch + 3])
-                     : "memory");
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t addr = prow + ((ch ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(codes[4 * ch]),
+                       "r"(codes[4 * ch + 1]), "r"(codes[4 * ch + 2]), "r"(codes[4 * ch + 3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        // the row's four block scales, on the sub-partition's diagonal column
+        tmem_st_32x32b_x1(trow + C::T_PSF + 4 * b + q, sfw);
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(b));
       }
-      fence_proxy_async_smem();
-      // the row's four block scales, on the sub-partition's diagonal column
-      tmem_st_32x32b_x1(trow + C::T_PSF + 4 * b + q, sfw);
-      tc_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full(b));
     }
-    // epilogue: O / rowsum -> bf16
-    if (ok && mbar_wait_bounded(o_full, 0)) {
+    // epilogue: O / (row sum of the quantised weights, O's column 128) ->
+    // bf16; warpgroup G writes columns [64 G, 64 G + 64)
+    if (__all_sync(0xffffffffu, ok && mbar_wait_bounded(o_full, 0))) {
       tc_fence_after();
-#pragma unroll
-      for (int i = 0; i < kAttD / 32; ++i) tmem_ld_32x32b_x32_nowait(trow + C::T_O + 32 * i, u + 32 * i);
+      tmem_ld_32x32b_x32_nowait(trow + C::T_O + 64 * G, u);
+      tmem_ld_32x32b_x32_nowait(trow + C::T_O + 64 * G + 32, u + 32);
+      uint32_t lsum = tmem_ld_32x32b_x1_nowait(trow + C::T_O + kAttD);
       tc_wait_ld();
+      reg_fence32(u);
+      reg_fence32(u + 32);
+      asm volatile("" : "+r"(lsum)::"memory");
+      const float inv_l = 1.0f / __uint_as_float(lsum);
+      uint4* dst = reinterpret_cast<uint4*>(args.out + (static_cast<int64_t>(qrow0) + r) * kAttD + 64 * G);
 #pragma unroll
-      for (int i = 0; i < kAttD / 32; ++i) reg_fence32(u + 32 * i);
-      const float inv_l = 1.0f / l;
-      uint4* dst = reinterpret_cast<uint4*>(args.out + (static_cast<int64_t>(qrow0) + r) * kAttD);
-#pragma unroll
-      for (int i = 0; i < kAttD / 8; ++i) {
+      for (int i = 0; i < 8; ++i) {
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -358,11 +492,14 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
 
 // V [heads][tokens][128] bf16 -> V^T MXFP8 codes [heads * 128][tokens] and
 // scales (rows heads * 128, tokens / 32 scale columns, swizzled), quantised
-// along tokens.  One CTA per (head, 128-token block); thread (c, blk)
-// quantises channel c over tokens [32 blk, 32 blk + 32) of the block.
-__global__ void __launch_bounds__(512) quantize_mxfp8_vt_kernel(const __nv_bfloat16* __restrict__ v, int heads,
-                                                              int tokens, uint8_t* __restrict__ codes,
-                                                              uint8_t* __restrict__ sf) {
+// along tokens.  One CTA per (head, 128-token block), 256 threads: thread
+// (p = tid % 64, blk = tid / 64) quantises channels 2p and 2p + 1 over tokens
+// [32 blk, 32 blk + 32) of the block, reading the staged tile as bf16 pairs
+// (a warp reads 128 contiguous bytes of a token row).
+constexpr int kVtThreads = 256;
+__global__ void __launch_bounds__(kVtThreads) quantize_mxfp8_vt_kernel(const __nv_bfloat16* __restrict__ v, int heads,
+                                                                     int tokens, uint8_t* __restrict__ codes,
+                                                                     uint8_t* __restrict__ sf) {
   __shared__ __align__(16) __nv_bfloat16 tile[kAttTile][kAttD];
   grid_dep_wait();
   grid_dep_launch();
@@ -370,28 +507,38 @@ __global__ void __launch_bounds__(512) quantize_mxfp8_vt_kernel(const __nv_bfloa
   const int h = blockIdx.x / nkb, t0 = (blockIdx.x % nkb) * kAttTile;
   const uint4* src = reinterpret_cast<const uint4*>(v + (static_cast<int64_t>(h) * tokens + t0) * kAttD);
   uint4* stile = reinterpret_cast<uint4*>(&tile[0][0]);
-  for (int i = threadIdx.x; i < kAttTile * kAttD / 8; i += blockDim.x) stile[i] = ldg_nc_v4(src + i);
+#pragma unroll
+  for (int i = 0; i < kAttTile * kAttD / 8 / kVtThreads; ++i)
+    stile[threadIdx.x + i * kVtThreads] = ldg_nc_v4(src + threadIdx.x + i * kVtThreads);
   __syncthreads();
-  const int c = threadIdx.x & (kAttD - 1), blk = threadIdx.x >> 7;
-  float f[32];
-  float bmax = 0.0f;
+  const int p = threadIdx.x & 63, blk = threadIdx.x >> 6;
+  float f0[32], f1[32];
+  float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    f[i] = __bfloat162float(tile[32 * blk + i][c]);
-    bmax = fmaxf(bmax, fabsf(f[i]));
+    const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&tile[32 * blk + i][2 * p]);
+    f0[i] = __low2float(pr);
+    f1[i] = __high2float(pr);
+    m0 = fmaxf(m0, fabsf(f0[i]));
+    m1 = fmaxf(m1, fabsf(f1[i]));
   }
-  int X = -127;
-  if (bmax > 0.0f) X = min(max(floor_log2_f32(bmax) - 8, -127), 127);  // OCP floor rule
-  const float mult = exp2_int(-X);
-  uint32_t w[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    w[i] = cvt_e4m3x2(f[4 * i] * mult, f[4 * i + 1] * mult) | (cvt_e4m3x2(f[4 * i + 2] * mult, f[4 * i + 3] * mult) << 16);
-  const int64_t row = static_cast<int64_t>(h) * kAttD + c;
-  uint4* dst = reinterpret_cast<uint4*>(codes + row * tokens + t0 + 32 * blk);
-  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  sf[sf_offset(row, (t0 >> 5) + blk, tokens >> 7)] = static_cast<uint8_t>(X + 127);
+  for (int ch = 0; ch < 2; ++ch) {
+    const float* f = ch == 0 ? f0 : f1;
+    const float bmax = ch == 0 ? m0 : m1;
+    int X = -127;
+    if (bmax > 0.0f) X = min(max(floor_log2_f32(bmax) - 8, -127), 127);  // OCP floor rule
+    const float mult = exp2_int(-X);
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      w[i] = cvt_e4m3x2(f[4 * i] * mult, f[4 * i + 1] * mult) | (cvt_e4m3x2(f[4 * i + 2] * mult, f[4 * i + 3] * mult) << 16);
+    const int64_t row = static_cast<int64_t>(h) * kAttD + 2 * p + ch;
+    uint4* dst = reinterpret_cast<uint4*>(codes + row * tokens + t0 + 32 * blk);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    sf[sf_offset(row, (t0 >> 5) + blk, tokens >> 7)] = static_cast<uint8_t>(X + 127);
+  }
   // rows heads * 128 are a multiple of 128: no scale padding to clear
 }
 

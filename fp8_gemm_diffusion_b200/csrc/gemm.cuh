@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(GemmCfg<F, BN>::THREADS, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mt = tile % m_tiles, nt = tile / m_tiles;
       const int m0 = mt * C::BM, n0 = nt * BN;
-      if (!mbar_wait_bounded(tfull_bar(acc), acc_phase)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(acc), acc_phase))) break;  // tcgen05.ld is warp-collective
       tc_fence_after();
       const int row0 = m0 + q * 32;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;

@@ -449,7 +449,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
       int sp = 0;               // A/B stage of g - NSF (the last user of set n)
       uint32_t rph = 0, spph = 0;
       for (int g = 0; g < total_kb; ++g) {
-        if (!mbar_wait_bounded(sf_full_bar(r), rph)) break;
+        // the tcgen05.st below is warp-collective: the warp leaves as a whole
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(sf_full_bar(r), rph))) break;
         const uint32_t slot = sf_base + r * C::SF_SLOT_BYTES;
         uint32_t va[NA], vb[NB * 4];
 #pragma unroll
@@ -467,7 +468,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
         // completed.  NSF <= STAGES, so the full barrier of stage g - STAGES
         // has completed too, and the arrival below counts towards stage g.
         if (g >= C::NSF) {
-          if (!mbar_wait_bounded(empty_bar(sp), spph)) break;
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(empty_bar(sp), spph))) break;
           if (++sp == S) { sp = 0; spph ^= 1u; }
         }
         tc_fence_after();
@@ -538,7 +539,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<F, BN>::THRE
           }
         }
       }
-      if (!mbar_wait_bounded(tfull_bar, i_tile & 1)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar, i_tile & 1))) break;  // tcgen05.ld is warp-collective
       tc_fence_after();
       // all of this warp's accumulator columns into registers, then release the accumulator
       uint32_t r[C::EPI_COLS];

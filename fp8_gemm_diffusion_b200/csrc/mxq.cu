@@ -254,8 +254,13 @@ mxq_status launch_quant_nvfp4_fused(const void* x, int64_t rows, int64_t k, int6
 
 mxq_status launch_quant_mxfp8(const void* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
                               uint8_t* sf, cudaStream_t s, int sms, int rceil = 0) {
-  cudaError_t e = launch_pdl(mxq::quantize_mxfp8_kernel, dim3(quant_grid(rows, sms)),
-                             dim3(mxq::kQuantThreads), 0, s, static_cast<const __nv_bfloat16*>(x),
+  // one thread per 32-element block, up to 8 CTAs per SM, grid-stride beyond
+  const int64_t nblk = rows * (k >> 5);
+  int64_t grid = (nblk + mxq::kMxThreads - 1) / mxq::kMxThreads;
+  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
+  if (grid < 1) grid = 1;
+  cudaError_t e = launch_pdl(mxq::quantize_mxfp8_kernel, dim3(static_cast<unsigned>(grid)),
+                             dim3(mxq::kMxThreads), 0, s, static_cast<const __nv_bfloat16*>(x),
                              static_cast<int>(rows), static_cast<int>(k), ld, codes, sf, rceil);
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
@@ -862,7 +867,7 @@ mxq_status mxq_attention_mxfp8(const void* q, const void* k, const void* v, int6
   if ((st = launch_quant_mxfp8(q, rows, d, d, base + l.q_codes, base + l.q_sf, s, sms)) != MXQ_OK) return st;
   if ((st = launch_quant_mxfp8(k, rows, d, d, base + l.k_codes, base + l.k_sf, s, sms)) != MXQ_OK) return st;
   const int grid = static_cast<int>(heads * (tokens / mxq::kAttTile));
-  cudaError_t e = launch_pdl(mxq::quantize_mxfp8_vt_kernel, dim3(grid), dim3(512), 0, s,
+  cudaError_t e = launch_pdl(mxq::quantize_mxfp8_vt_kernel, dim3(grid), dim3(mxq::kVtThreads), 0, s,
                              static_cast<const __nv_bfloat16*>(v), static_cast<int>(heads),
                              static_cast<int>(tokens), base + l.v_codes, base + l.v_sf);
   if (e != cudaSuccess) return cuda_fail(e);

@@ -63,6 +63,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase (mbarrier.test_wait): for a thread that polls
+// several barriers and serves whichever completes first.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Returns false
 // (and records kErrTimeout) when the wait runs out.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
@@ -405,11 +419,19 @@ __device__ __forceinline__ void reg_fence32(uint32_t* r) {
                  "+r"(r[30]), "+r"(r[31])::"memory");
 }
 
-// Store 4 consecutive 32-bit columns of this warp's 32 lanes.
+// Store one 32-bit column of this warp's 32 lanes.
 __device__ __forceinline__ void tmem_st_32x32b_x1(uint32_t taddr, uint32_t a) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(a) : "memory");
 }
 
+// Load one 32-bit column of this warp's 32 lanes (no wait; see tc_wait_ld).
+__device__ __forceinline__ uint32_t tmem_ld_32x32b_x1_nowait(uint32_t taddr) {
+  uint32_t a;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(a) : "r"(taddr) : "memory");
+  return a;
+}
+
+// Store 4 consecutive 32-bit columns of this warp's 32 lanes.
 __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c,
                                                   uint32_t d) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a),
@@ -504,6 +526,18 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bo
       : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
       : "memory");
   return r != 0;
+}
+
+
+// Named barrier `id` (1..15) over `nthreads` threads (whole warps), split in
+// a producer side that only signals (bar.arrive) and a consumer side that
+// waits (bar.sync); shared-memory writes before the arrive are visible
+// after the sync.
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 }  // namespace mxq

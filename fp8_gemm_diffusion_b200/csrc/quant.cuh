@@ -506,52 +506,60 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 }
 
 // -------------------------------------------------------------- MXFP8
-__global__ void __launch_bounds__(kQuantThreads)
+// bmax > 1.75 * 2^floor(log2 bmax), exactly, for a positive finite fp32 (the
+// ceiling rule's "one more" decision: 448 * 2^(e - 8) = 1.75 * 2^e).  A
+// normal value compares its fraction bits with 0.75 (0x600000); a subnormal
+// m * 2^-149 compares m with 1.75 * 2^floor(log2 m) in integers.
+__device__ __forceinline__ bool above_1p75(float bmax) {
+  const uint32_t b = __float_as_uint(bmax);
+  if (b >= 0x00800000u) return (b & 0x7FFFFFu) > 0x600000u;
+  const uint32_t m = b & 0x7FFFFFu;
+  const int fl = 31 - __clz(m);
+  return 4u * m > (7u << fl);
+}
+
+// One thread per 32-element block: 64 bytes in (four 16-byte loads), 32
+// bytes of codes out (two 16-byte stores) and the block's scale byte;
+// consecutive threads take consecutive blocks of a row, then the next row,
+// so a warp reads and writes contiguous memory for any k.
+constexpr int kMxThreads = 256;
+__global__ void __launch_bounds__(kMxThreads)
     quantize_mxfp8_kernel(const __nv_bfloat16* __restrict__ x, int rows, int k, int64_t ld,
                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf, int rceil) {
   grid_dep_wait();
   grid_dep_launch();
-  const int lane = threadIdx.x & 31;
-  const int warps = gridDim.x * (kQuantThreads / 32);
-  const int vpr = k >> 3;  // multiple of 16: k is a multiple of 128
+  const int bpr = k >> 5;  // blocks per row
   const int c4 = k >> 7;
-  for (int r = blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
-    const __nv_bfloat16* row = x + static_cast<int64_t>(r) * ld;
-    uint2* crow = reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * k);
-    for (int v0 = lane; v0 - lane < vpr; v0 += 32 * kQuantUnroll) {
-      uint4 u[kQuantUnroll];
+  const int64_t nblk = static_cast<int64_t>(rows) * bpr;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * kMxThreads + threadIdx.x; t < nblk;
+       t += static_cast<int64_t>(gridDim.x) * kMxThreads) {
+    const int r = static_cast<int>(t / bpr), c = static_cast<int>(t - static_cast<int64_t>(r) * bpr);
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ld + 32 * c);
+    uint4 u[4];
 #pragma unroll
-      for (int j = 0; j < kQuantUnroll; ++j) {
-        const int v = v0 + 32 * j;
-        u[j] = v < vpr ? ldg_nc_v4(row + v * 8) : make_uint4(0, 0, 0, 0);
-      }
+    for (int i = 0; i < 4; ++i) u[i] = ldg_nc_v4(src + i);
+    float f[32];
 #pragma unroll
-      for (int j = 0; j < kQuantUnroll; ++j) {
-        const int v = v0 + 32 * j;
-        if (v - lane >= vpr) break;  // warp-uniform
-        float f[8];
-        bf16x8_to_f32(u[j], f);
-        float bmax = absmax8(f);
-        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 1));
-        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 2));  // 32-element block
-        int X = -127;
-        if (bmax > 0.0f) {
-          int e = floor_log2_f32(bmax) - 8;
-          // ceiling rule: the smallest X with bmax <= 448 * 2^X, i.e. one more
-          // when bmax > 1.75 * 2^(e + 8) (exact in double)
-          if (rceil && static_cast<double>(bmax) > ldexp(1.75, e + 8)) e += 1;
-          X = min(max(e, -127), 127);
-        }
-        const float mult = exp2_int(-X);
-        uint2 out;
-        out.x = cvt_e4m3x2(f[0] * mult, f[1] * mult) | (cvt_e4m3x2(f[2] * mult, f[3] * mult) << 16);
-        out.y = cvt_e4m3x2(f[4] * mult, f[5] * mult) | (cvt_e4m3x2(f[6] * mult, f[7] * mult) << 16);
-        if (v < vpr) {
-          crow[v] = out;
-          if ((v & 3) == 0) sf[sf_offset(r, v >> 2, c4)] = static_cast<uint8_t>(X + 127);
-        }
-      }
+    for (int i = 0; i < 4; ++i) bf16x8_to_f32(u[i], *reinterpret_cast<float(*)[8]>(f + 8 * i));
+    float bmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) bmax = fmaxf(bmax, fabsf(f[i]));
+    int X = -127;
+    if (bmax > 0.0f) {
+      // floor rule (OCP): X = floor(log2 bmax) - 8; ceiling rule: the smallest
+      // X with bmax <= 448 * 2^X, one more when bmax > 1.75 * 2^floor(log2 bmax)
+      const int e = floor_log2_f32(bmax) - 8 + ((rceil && above_1p75(bmax)) ? 1 : 0);
+      X = min(max(e, -127), 127);
     }
+    const float mult = exp2_int(-X);
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      w[i] = cvt_e4m3x2(f[4 * i] * mult, f[4 * i + 1] * mult) | (cvt_e4m3x2(f[4 * i + 2] * mult, f[4 * i + 3] * mult) << 16);
+    uint4* dst = reinterpret_cast<uint4*>(codes + static_cast<int64_t>(r) * k + 32 * c);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    sf[sf_offset(r, c, c4)] = static_cast<uint8_t>(X + 127);
   }
   zero_sf_padding(sf, rows, k >> 5);
 }

@@ -316,14 +316,17 @@ mxq_status mxq_linear_noalloc(const mxq_weight* w, const void* x_bf16, int64_t M
  *   Q, K -> MXFP8 (E4M3 codes, one power-of-two scale per token and per 32
  *   channels), V -> MXFP8 of V^T (per channel and per 32 tokens);
  *   S = deq(Q) deq(K)^T on the tensor cores (fp32); softmax along keys with
- *   scale tau, exact (row maximum first, then the weights
- *   E = 2^((S - max) tau log2 e) in fp32); E -> MXFP8 along keys (ceiling
- *   scale rule, no saturation); O = deq(E) deq(V^T)^T / rowsum(E) on the
- *   tensor cores (fp32), bf16 out.
- * Accuracy: |O - O_exact| <= 0.07 * T + 1e-6 per element, with O_exact the
- * float64 attention on the quantised Q, K, V and T = sum over 32-key blocks
- * of (the block's softmax mass) x (the block's max |V|) -- the rounding of E
- * to E4M3 (at most 2^-4 of each weight) dominates.
+ *   scale tau through the weights E = 2^(t - m) in fp32, t = S tau log2 e,
+ *   m an integer (any integer gives the same codes: a power-of-two factor
+ *   moves only a block's shared exponent; the kernel takes a running
+ *   maximum in one pass over the keys); E -> MXFP8 along keys (ceiling scale
+ *   rule, no saturation); O = deq(E) deq(V^T)^T / rowsum(deq(E)) on the
+ *   tensor cores (fp32; each query row divided by the sum of its quantised
+ *   weights, the per-token correction of their rounding), bf16 out.
+ * Accuracy: |O - O_exact| <= 0.14 * T + 2^-11 * max_j |V[j, c]| + 1e-6 per
+ * element, with O_exact the float64 attention on the quantised Q, K, V and
+ * T = sum_j P[i, j] |V[j, c]| -- the rounding of E to E4M3 (at most 2^-4 of
+ * each weight, twice through the renormalisation) dominates.
  *
  * mxq_attention_workspace_bytes - device bytes mxq_attention_mxfp8 needs
  * (the quantised Q, K, V^T and their scales); 0 for unsupported arguments.

@@ -3,16 +3,22 @@
 Each output is compared with the float64 oracle on the same quantised Q, K, V
 (oracle/attention.py):
 - every element within the derived worst-case bound of the exact
-  softmax-weighted sum (0.07 T + 2^-12 max|V| + 1e-6, T = sum_j P_j |V_j|;
+  softmax-weighted sum (0.14 T + 2^-11 max|V| + 1e-6, T = sum_j P_j |V_j|;
   the rounding of the weights to E4M3 dominates it);
-- at least 99.9 % of the elements within 2e-3 * T + 1e-6 (the GEMM's rule)
-  of the oracle doing the kernel's own rounding of the weights (ceiling-rule
-  MXFP8 of E = exp(S - max)): only weights that land on the other side of a
-  rounding boundary (fp32 vs float64 logits and exponentials) differ;
+- at least 99.9 % of the elements within 2^-9 |O_q| + 2e-3 T + 1e-6 (the bf16
+  output's rounding plus the GEMM's rule) of the oracle doing the kernel's
+  own rounding of the weights (ceiling-rule MXFP8 of E = 2^(t - m), m an
+  integer): only weights that land on the other side of a rounding boundary
+  (fp32 vs float64 logits and exponentials) differ.  With logits in the
+  hundreds the tensor cores' error in S moves E itself (through the row sum
+  for one dominant key per row, the peaked case, which the bf16 term of the
+  bound covers); for logits that rise along the keys, where several large
+  weights share a row, 99 %;
 - the median element within 1 % of that result (no systematic deviation).
 Shapes: one key block, several, a FLUX-sized call (24 heads x 4608 tokens,
-sampled rows), a peaked softmax (one dominant key per query), an explicit
-softmax scale, and two calls in a row giving the same bits.
+sampled rows), a peaked softmax (one dominant key per query), logits that
+rise along the keys (the running normaliser moves at every key block) and
+fall, an explicit softmax scale, and two calls in a row giving the same bits.
 """
 
 import numpy as np
@@ -35,7 +41,7 @@ def _run(Q, K, V, tau=0.0):
     return out
 
 
-def _check(Q, K, V, out, heads=None, rows=None, tau=None):
+def _check(Q, K, V, out, heads=None, rows=None, tau=None, min_tight=0.999):
     H = Q.shape[0]
     for h in (range(H) if heads is None else heads):
         O, Terr, Oq, vmax = A.attention_ref(Q[h], K[h], V[h], rows=rows, tau=tau)
@@ -45,7 +51,7 @@ def _check(Q, K, V, out, heads=None, rows=None, tau=None):
         ok = A.within_att_tol(og, O, Terr, vmax)
         assert ok.all(), f"head {h}: {np.count_nonzero(~ok)} outputs past the derived bound"
         tight = A.within_att_tight(og, Oq, Terr)
-        assert tight.mean() >= 0.999, f"head {h}: only {tight.mean():.5f} of the outputs within 2e-3 T of O_q"
+        assert tight.mean() >= min_tight, f"head {h}: only {tight.mean():.5f} of the outputs within the sharp bound"
         # no systematic deviation: the typical element is as close to O_q as
         # its bf16 rounding (2^-9) and a few rounding-boundary weights allow
         rel = np.abs(og - Oq) / (np.abs(Oq) + 1e-6)
@@ -75,6 +81,24 @@ def test_attention_peaked_softmax():
     K = (Q.float() * 8.0).bfloat16()
     out = _run(Q, K, V)
     _check(Q, K, V, out)
+
+
+def test_attention_rising_logits_raise_the_running_maximum():
+    # the keys grow along the sequence in the queries' direction: every key
+    # block's maximum logit is about 10 (in log2 units) above the previous
+    # block's, so the kernel raises its normaliser and rescales the output
+    # accumulator at every block; the falling order never does
+    H, T, d = 1, 640, 128
+    g = torch.Generator().manual_seed(21)
+    u = torch.randn(d, generator=g)
+    Q = (u + 0.1 * torch.randn(T, d, generator=g)).unsqueeze(0)
+    ramp = torch.linspace(0.0, 3.2, T).unsqueeze(1)
+    K = (ramp * u + 0.1 * torch.randn(T, d, generator=g)).unsqueeze(0)
+    V = torch.randn(1, T, d, generator=g)
+    for Kx in (K, K.flip(1)):
+        Qb, Kb, Vb = Q.bfloat16(), Kx.bfloat16(), V.bfloat16()
+        out = _run(Qb, Kb, Vb)
+        _check(Qb, Kb, Vb, out, min_tight=0.99)
 
 
 def test_attention_explicit_tau_and_repeatability():

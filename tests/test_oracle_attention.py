@@ -4,9 +4,11 @@ Pinned against: explicit loops with math.exp on tiny inputs (no numpy
 softmax or matmul), softmax invariants, closed forms (equal keys give the
 mean of the values, equal values pass through, two keys give the logistic
 function), inputs that MXFP8 represents exactly (the quantised attention
-must then equal the plain one), and the derived error bound (it holds for
-the rounding of the weights, and the sharp check rejects a planted scale
-mistake and a dropped key block).
+must then equal the plain one), the power-of-two normaliser (explicit
+loops; an integer shift of it leaves every code and the dequantised result
+up to that power of two unchanged), and the derived error bound (it holds
+for the rounding of the weights, and the sharp check rejects a planted
+scale mistake and a dropped key block).
 """
 
 import math
@@ -16,6 +18,7 @@ import pytest
 import torch
 
 from oracle import attention as A
+from oracle import quant as Qz
 
 
 def _bf16(x):
@@ -97,6 +100,20 @@ def test_equal_values_pass_through():
     assert np.allclose(O, np.tile(v.astype(np.float64), (T, 1)), atol=1e-14)
 
 
+def test_quantised_weights_renormalise_a_constant_value_exactly():
+    # the division by the sum of the quantised weights: with every key's value
+    # equal (and exactly representable) the quantised path returns it exactly,
+    # whatever the rounding of the weights; a division by the unquantised sum
+    # would be off by the weights' mean rounding error
+    rng = np.random.default_rng(9)
+    T, d = 96, 32
+    Q, K = (rng.normal(size=(T, d)).astype(np.float32) * 2 for _ in range(2))
+    v = np.float32(2.0 ** -3) * rng.integers(-7, 8, size=d).astype(np.float32)
+    V = np.tile(v, (T, 1))
+    _, _, Oq, _ = A.attention_ref(_bf16(Q), _bf16(K), _bf16(V))
+    assert np.array_equal(Oq, np.tile(v.astype(np.float64), (T, 1)))
+
+
 def test_two_key_closed_form():
     # plain attention, two keys: p = sigmoid(tau (s0 - s1))
     Q = np.array([[1.0, 2.0]])
@@ -107,6 +124,35 @@ def test_two_key_closed_form():
     p = 1 / (1 + math.exp(-tau * (d0 - d1)))
     want = p * V[0] + (1 - p) * V[1]
     assert np.allclose(A.attention_plain(Q, K, V)[0], want, atol=1e-14)
+
+
+def test_pow2_weights_match_explicit_loops():
+    t = np.array([[0.25, 3.5, -1.0], [-7.75, -7.5, -9.0]])
+    E = A.weights_pow2(t)
+    for i in range(2):
+        m = math.ceil(max(t[i]))
+        for j in range(3):
+            assert E[i, j] == 2.0 ** (t[i, j] - m)
+    # the largest weight of a row lies in (1/2, 1]
+    rng = np.random.default_rng(7)
+    E = A.weights_pow2(rng.normal(size=(16, 64)) * 5)
+    assert np.all(E.max(axis=1) <= 1.0) and np.all(E.max(axis=1) > 0.5)
+
+
+def test_power_of_two_normaliser_leaves_codes_and_result_unchanged():
+    # the reading's claim: shifting m by an integer k scales every block by
+    # 2^-k, moves each ceiling-rule shared exponent by -k and keeps every code
+    rng = np.random.default_rng(8)
+    t = rng.normal(size=(8, 256)) * 3
+    E0 = A.weights_pow2(t).astype(np.float32)
+    for k in (-8, -3, 5):
+        Ek = A.weights_pow2(t, shift=k).astype(np.float32)
+        q0 = Qz.quantize_mxfp8(E0, scale_rule="rceil")
+        qk = Qz.quantize_mxfp8(Ek, scale_rule="rceil")
+        assert np.array_equal(q0["codes"], qk["codes"])
+        d0 = Qz.dequant_mxfp8(q0["codes"], q0["sf"])
+        dk = Qz.dequant_mxfp8(qk["codes"], qk["sf"])
+        assert np.array_equal(dk, d0 * 2.0 ** -k)
 
 
 def test_bounds_hold_for_the_weight_rounding_and_reject_planted_mistakes():
