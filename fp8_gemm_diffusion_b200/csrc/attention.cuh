@@ -27,15 +27,17 @@
 // rescaled with O and divided out at the end.
 //
 // One CTA per (head, 128-query tile), 12 warps:
-//   warp 0      TMA producer: the Q tile and its scales once, then a ring of
-//               key blocks (K, V^T and their 512-byte scale chunks);
-//   warp 1      tensor memory; one lane issues the scale copies (tcgen05.cp)
-//               and the MMAs: S = Q K^T of block j into S buffer j % 2, and
-//               O += Eq V^T of block j once its weights are in place;
+//   warp 0      TMA producer of the Q tile and of K (and scales) per block;
+//   warp 2      TMA producer of V^T (and scales) per block;
+//   warp 1      tensor memory; one lane issues S = Q K^T of block j into S
+//               buffer j % 2 (with the scale copies, tcgen05.cp);
+//   warp 3      one lane issues O += Eq V^T of block j once its weights are
+//               in place;
 //   warps 4-7   softmax of the even key blocks, warps 8-11 of the odd ones
 //               (tensor-memory sub-partition warp % 4, one query row per
 //               thread): the two warpgroups work on consecutive blocks at
-//               the same time, each hiding the other's waits.  Per block:
+//               the same time (two warps per sub-partition keep the
+//               exponential unit busy).  Per block:
 //               block maxima, the normaliser (taken over from the other
 //               warpgroup's previous block through shared memory and raised
 //               if needed), weights, MXFP8 codes of E into shared memory
@@ -121,6 +123,18 @@ __device__ __forceinline__ int mx_ceil_exponent_normal(float bmax) {
   return min(max(X, -127), 127);
 }
 
+// Four fp32 -> four E4M3 bytes packed into 32 bits, a in the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
+
 // Instruction descriptor of an M = 128 kind::mxf8f6f4 MMA (E4M3 x E4M3,
 // UE8M0 scales) with separate scale-byte selectors for A and B.
 __device__ __forceinline__ uint32_t idesc_mxfp8_m128(int n, uint32_t a_id, uint32_t b_id) {
@@ -152,17 +166,23 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* const base_ptr = smem_raw + (base - raw_addr);
   const uint32_t bar = base + C::OFF_BAR;
-  // barriers: q_full, kv_full[4], kv_empty[4], s_full[2], s_free[2], p_full[2], p_free[2], o_full
+  // barriers: q_full, k_full[4], k_empty[4], v_full[4], v_empty[4], s_full[2], s_free[2],
+  // p_full[2], p_free[2], o_full, qk_drain.  K and V^T of a stage have their own
+  // barriers: K is free once S of its block is computed, long before V^T
+  // is, so the K ring runs ahead of the V^T ring.
   const uint32_t q_full = bar;
-  auto kv_full = [&](int s) { return bar + 8u + 8u * s; };
-  auto kv_empty = [&](int s) { return bar + 8u + 8u * (kAttStages + s); };
-  auto s_full = [&](int b) { return bar + 8u + 8u * (2 * kAttStages + b); };
-  auto s_free = [&](int b) { return bar + 8u + 8u * (2 * kAttStages + 2 + b); };
-  auto p_full = [&](int b) { return bar + 8u + 8u * (2 * kAttStages + 4 + b); };
-  auto p_free = [&](int b) { return bar + 8u + 8u * (2 * kAttStages + 6 + b); };
-  const uint32_t o_full = bar + 8u + 8u * (2 * kAttStages + 8);
-  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_BAR + 8 * (2 * kAttStages + 10));
-  static_assert(8 * (2 * kAttStages + 10) + 4 <= C::BAR_BYTES, "barrier area");
+  auto k_full = [&](int s) { return bar + 8u + 8u * s; };
+  auto k_empty = [&](int s) { return bar + 8u + 8u * (kAttStages + s); };
+  auto v_full = [&](int s) { return bar + 8u + 8u * (2 * kAttStages + s); };
+  auto v_empty = [&](int s) { return bar + 8u + 8u * (3 * kAttStages + s); };
+  auto s_full = [&](int b) { return bar + 8u + 8u * (4 * kAttStages + b); };
+  auto s_free = [&](int b) { return bar + 8u + 8u * (4 * kAttStages + 2 + b); };
+  auto p_full = [&](int b) { return bar + 8u + 8u * (4 * kAttStages + 4 + b); };
+  auto p_free = [&](int b) { return bar + 8u + 8u * (4 * kAttStages + 6 + b); };
+  const uint32_t o_full = bar + 8u + 8u * (4 * kAttStages + 8);
+  const uint32_t qk_drain = bar + 8u + 8u * (4 * kAttStages + 9);  // the S thread's last MMAs done
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_BAR + 8 * (4 * kAttStages + 11));
+  static_assert(8 * (4 * kAttStages + 11) + 4 <= C::BAR_BYTES, "barrier area");
   constexpr int NSOFT = 4;  // warps of one softmax warpgroup (the one that owns S / P buffer b)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -174,8 +194,10 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kAttStages; ++s) {
-      mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full(b), 1);
@@ -184,6 +206,7 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
       mbar_init(p_free(b), 1);
     }
     mbar_init(o_full, 1);
+    mbar_init(qk_drain, 1);
     fence_barrier_init();
     prefetch_tmap(&tmap_q);
     prefetch_tmap(&tmap_k);
@@ -214,25 +237,33 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
 
   if (warp < C::SOFT_WARP0) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_CTRL));
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ producers
+    // warp 0: the Q tile, then K and its scales per key block; warp 2: V^T
+    // and its scales per key block, each into its part of the stage ring
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, C::TILE_BYTES + 512);
-      tma_load_2d(base, &tmap_q, q_full, 0, qrow0);
-      bulk_load(base + C::OFF_QSF, args.q_sf + static_cast<int64_t>(qrow0 / 128) * 512, 512, q_full);
+      const bool is_k = warp == 0;
+      if (is_k) {
+        mbar_arrive_expect_tx(q_full, C::TILE_BYTES + 512);
+        tma_load_2d(base, &tmap_q, q_full, 0, qrow0);
+        bulk_load(base + C::OFF_QSF, args.q_sf + static_cast<int64_t>(qrow0 / 128) * 512, 512, q_full);
+      }
       int s = 0, issued = 0;
       uint32_t ph = 0;
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait_bounded(kv_empty(s), ph ^ 1u)) { ok = false; break; }
+        if (!mbar_wait_bounded(is_k ? k_empty(s) : v_empty(s), ph ^ 1u)) { ok = false; break; }
         const uint32_t st = base + C::OFF_STAGE + s * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(kv_full(s), 2u * (C::TILE_BYTES + 512));
-        const int krow = h * T + kb * kAttTile;
-        tma_load_2d(st, &tmap_k, kv_full(s), 0, krow);
-        bulk_load(st + C::ST_KSF, args.k_sf + static_cast<int64_t>(krow / 128) * 512, 512, kv_full(s));
-        tma_load_2d(st + C::TILE_BYTES, &tmap_v, kv_full(s), kb * kAttTile, h * kAttD);
-        bulk_load(st + C::ST_VSF, args.v_sf + (static_cast<int64_t>(h) * nkb + kb) * 512, 512,
-                  kv_full(s));
+        if (is_k) {
+          mbar_arrive_expect_tx(k_full(s), C::TILE_BYTES + 512);
+          const int krow = h * T + kb * kAttTile;
+          tma_load_2d(st, &tmap_k, k_full(s), 0, krow);
+          bulk_load(st + C::ST_KSF, args.k_sf + static_cast<int64_t>(krow / 128) * 512, 512, k_full(s));
+        } else {
+          mbar_arrive_expect_tx(v_full(s), C::TILE_BYTES + 512);
+          tma_load_2d(st + C::TILE_BYTES, &tmap_v, v_full(s), kb * kAttTile, h * kAttD);
+          bulk_load(st + C::ST_VSF, args.v_sf + (static_cast<int64_t>(h) * nkb + kb) * 512, 512, v_full(s));
+        }
         ++issued;
         if (++s == kAttStages) { s = 0; ph ^= 1u; }
       }
@@ -240,92 +271,75 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
         // let the loads already issued land before the CTA can exit
         for (int i = 0; i < kAttStages && i < issued; ++i) {
           if (--s < 0) { s = kAttStages - 1; ph ^= 1u; }
-          mbar_wait_bounded(kv_full(s), ph);
+          mbar_wait_bounded(is_k ? k_full(s) : v_full(s), ph);
         }
       }
-      mbar_wait_bounded(q_full, 0);
+      if (is_k) mbar_wait_bounded(q_full, 0);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two threads: warp 1 issues S = Q K^T (into the S buffers), warp 3 the
+    // second product O += Eq V^T (into O).  They write disjoint tensor memory
+    // and each product's inputs arrive through mbarriers, so the two need no
+    // order between them; each thread's own MMAs (one accumulator each) stay
+    // in issue order.  An MMA takes about a hundred cycles to issue, so one
+    // thread for both products became the limit.
     if (lane == 0) {
       bool ok = mbar_wait_bounded(q_full, 0);
       tc_fence_after();
-      if (ok) {
-        tc_cp_32x128b_warpx4(tmem + C::T_QSF, desc_sf_chunk(base + C::OFF_QSF));
+      if (warp == 1) {
+        if (ok) tc_cp_32x128b_warpx4(tmem + C::T_QSF, desc_sf_chunk(base + C::OFF_QSF));
+        const uint64_t qdesc = desc_kmajor_sw128(base);
+        for (int j = 0; j < nkb && ok; ++j) {
+          const int st_idx = j % kAttStages;
+          // K of block j has landed; the softmax has read S of block j - 2
+          if (!(ok = mbar_wait_bounded(k_full(st_idx), (j / kAttStages) & 1))) break;
+          if (!(ok = mbar_wait_bounded(s_free(j & 1), ((j >> 1) & 1) ^ 1u))) break;
+          tc_fence_after();
+          const uint32_t st = base + C::OFF_STAGE + st_idx * C::STAGE_BYTES;
+          tc_cp_32x128b_warpx4(tmem + C::T_KSF, desc_sf_chunk(st + C::ST_KSF));
+          const uint64_t kdesc = desc_kmajor_sw128(st);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t koff = static_cast<uint64_t>(2 * k);  // 32 bytes of d per MMA
+            mma_mxfp8(tmem + C::T_S + (j & 1) * kAttTile, qdesc + koff, kdesc + koff,
+                      idesc_mxfp8_m128(kAttTile, k, k), (tmem + C::T_QSF) | (static_cast<uint32_t>(k) << 30),
+                      (tmem + C::T_KSF) | (static_cast<uint32_t>(k) << 30), k > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full(j & 1));
+          tc_commit(k_empty(st_idx));
+        }
+        // every MMA / copy this thread issued must finish before tensor memory is freed
+        tc_commit(qk_drain);
+        mbar_wait_bounded(qk_drain, 0);
+      } else {
         // unit scales of the V^T extension rows (128-row group 1 of the B scales), once
         tc_cp_32x128b_warpx4(tmem + C::T_VSF + 4, desc_sf_chunk(base + C::OFF_ONESF));
-      }
-      const uint64_t qdesc = desc_kmajor_sw128(base);
-      // S[j % 2] = Q K^T of key block j (stage j % kAttStages); its scale
-      // chunk is copied first, behind the previous MMAs in this thread's order
-      auto issue_qk = [&](int j) {
-        tc_fence_after();
-        const uint32_t st = base + C::OFF_STAGE + (j % kAttStages) * C::STAGE_BYTES;
-        tc_cp_32x128b_warpx4(tmem + C::T_KSF, desc_sf_chunk(st + C::ST_KSF));
-        const uint64_t kdesc = desc_kmajor_sw128(st);
+        for (int j = 0; j < nkb && ok; ++j) {
+          const int b = j & 1, st_idx = j % kAttStages;
+          // the weights of block j are in place and its V^T has landed
+          if (!(ok = mbar_wait_bounded(p_full(b), (j >> 1) & 1))) break;
+          if (!(ok = mbar_wait_bounded(v_full(st_idx), (j / kAttStages) & 1))) break;
+          tc_fence_after();
+          const uint32_t st = base + C::OFF_STAGE + st_idx * C::STAGE_BYTES;
+          tc_cp_32x128b_warpx4(tmem + C::T_VSF, desc_sf_chunk(st + C::ST_VSF));
+          const uint64_t pdesc = desc_kmajor_sw128(base + C::OFF_P + b * C::TILE_BYTES);
+          const uint64_t vdesc = desc_kmajor_sw128(st + C::TILE_BYTES);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t koff = static_cast<uint64_t>(2 * k);  // 32 bytes of d per MMA
-          mma_mxfp8(tmem + C::T_S + (j & 1) * kAttTile, qdesc + koff, kdesc + koff,
-                    idesc_mxfp8_m128(kAttTile, k, k), (tmem + C::T_QSF) | (static_cast<uint32_t>(k) << 30),
-                    (tmem + C::T_KSF) | (static_cast<uint32_t>(k) << 30), k > 0 ? 1u : 0u);
-        }
-        tc_commit(s_full(j & 1));
-      };
-      // O += Eq V^T of key block j; MMA k covers keys [32 k, 32 k + 32),
-      // scale byte k of the row's word
-      auto issue_pv = [&](int j) {
-        const int b = j & 1, st_idx = j % kAttStages;
-        tc_fence_after();
-        const uint32_t st = base + C::OFF_STAGE + st_idx * C::STAGE_BYTES;
-        tc_cp_32x128b_warpx4(tmem + C::T_VSF, desc_sf_chunk(st + C::ST_VSF));
-        const uint64_t pdesc = desc_kmajor_sw128(base + C::OFF_P + b * C::TILE_BYTES);
-        const uint64_t vdesc = desc_kmajor_sw128(st + C::TILE_BYTES);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t koff = static_cast<uint64_t>(2 * k);  // 32 keys per MMA
-          mma_mxfp8(tmem + C::T_O, pdesc + koff, vdesc + koff, idesc_mxfp8_m128(C::PV_N, k, k),
-                    (tmem + C::T_PSF + 4 * b) | (static_cast<uint32_t>(k) << 30),
-                    (tmem + C::T_VSF) | (static_cast<uint32_t>(k) << 30), (j > 0 || k > 0) ? 1u : 0u);
-        }
-        tc_commit(p_free(b));
-        tc_commit(kv_empty(st_idx));
-      };
-      // Serve whichever is ready: S of block jq (its K has landed and the
-      // softmax has read S of block jq - 2 from the same buffer) or the
-      // product of block jp (its weights are in place).  The two warpgroups
-      // then run independently; the products stay in block order, which the
-      // rescaling of O relies on.  A stretch of 2 s without progress ends
-      // the loop with a timeout.
-      int jq = 0, jp = 0;
-      uint32_t idle = 0;
-      uint64_t t_idle = 0;
-      while (ok && jp < nkb) {
-        bool did = false;
-        if (jq < nkb && mbar_test(kv_full(jq % kAttStages), (jq / kAttStages) & 1) &&
-            mbar_test(s_free(jq & 1), ((jq >> 1) & 1) ^ 1u)) {
-          issue_qk(jq++);
-          did = true;
-        }
-        if (jp < jq && mbar_test(p_full(jp & 1), (jp >> 1) & 1)) {
-          issue_pv(jp++);
-          did = true;
-        }
-        if (did) {
-          idle = 0;
-        } else if ((++idle & 255u) == 0u) {
-          const uint64_t now = globaltimer_ns();
-          if (idle == 256u) {
-            t_idle = now;
-          } else if (now - t_idle > kWaitLimitNs) {
-            record_error(kErrTimeout);
-            ok = false;
+          for (int k = 0; k < 4; ++k) {
+            // MMA k covers keys [32 k, 32 k + 32), scale byte k of the row's word
+            const uint64_t koff = static_cast<uint64_t>(2 * k);
+            mma_mxfp8(tmem + C::T_O, pdesc + koff, vdesc + koff, idesc_mxfp8_m128(C::PV_N, k, k),
+                      (tmem + C::T_PSF + 4 * b) | (static_cast<uint32_t>(k) << 30),
+                      (tmem + C::T_VSF) | (static_cast<uint32_t>(k) << 30), (j > 0 || k > 0) ? 1u : 0u);
           }
+          tc_commit(p_free(b));
+          tc_commit(v_empty(st_idx));
         }
+        tc_commit(o_full);
+        // every MMA / copy this thread issued must finish before tensor memory is freed
+        mbar_wait_bounded(o_full, 0);
       }
-      tc_commit(o_full);
-      // every MMA / copy issued above must finish before tensor memory is freed
-      mbar_wait_bounded(o_full, 0);
     }
   }
   } else {
@@ -372,6 +386,9 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
       }
       const bool raise = tmax > m + kAttRescale;
       const float m_new = raise ? ceilf(tmax) : m;
+      // hand the normaliser on at once: the other warpgroup's block j + 1
+      // runs its exponentials alongside these (two warps per sub-partition
+      // keep the exponential unit busy)
       if (j + 1 < nkb) {
         xm[r] = m_new;
         __syncwarp();
@@ -412,25 +429,25 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
       }
       m = m_new;
       // weights of the four 32-key blocks, their MXFP8 codes and scales (the
-      // row sum of the quantised weights comes out of the second product)
-      uint32_t codes[kAttTile / 4];
+      // row sum of the quantised weights comes out of the second product):
+      // the block exponents first, then all 128 exponentials in place
+      // (independent, back to back on the exponential unit), then the codes
+      float mx[4];
       uint32_t sfw = 0;
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) {
         const float emax = ex2_approx(fmaf(bm[blk], c, -m));
         const int X = mx_ceil_exponent_normal(emax);
-        const float mx = m + static_cast<float>(X);  // E / 2^X = 2^(t - m - X)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t* v = u + 32 * blk + 4 * i;
-          const float e0 = ex2_approx(fmaf(__uint_as_float(v[0]), c, -mx));
-          const float e1 = ex2_approx(fmaf(__uint_as_float(v[1]), c, -mx));
-          const float e2 = ex2_approx(fmaf(__uint_as_float(v[2]), c, -mx));
-          const float e3 = ex2_approx(fmaf(__uint_as_float(v[3]), c, -mx));
-          codes[8 * blk + i] = cvt_e4m3x2(e0, e1) | (cvt_e4m3x2(e2, e3) << 16);
-        }
+        mx[blk] = m + static_cast<float>(X);  // E / 2^X = 2^(t - m - X)
         sfw |= static_cast<uint32_t>(X + 127) << (8 * blk);
       }
+#pragma unroll
+      for (int i = 0; i < kAttTile; ++i) u[i] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(u[i]), c, -mx[i >> 5])));
+      uint32_t codes[kAttTile / 4];
+#pragma unroll
+      for (int i = 0; i < kAttTile / 4; ++i)
+        codes[i] = cvt_e4m3x4(__uint_as_float(u[4 * i]), __uint_as_float(u[4 * i + 1]), __uint_as_float(u[4 * i + 2]),
+                              __uint_as_float(u[4 * i + 3]));
       // the product of block j - 2 (this warpgroup's previous block) has read
       // this buffer and its scales
       ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(p_free(b), ((j >> 1) & 1) ^ 1u));
