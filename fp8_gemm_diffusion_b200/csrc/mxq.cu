@@ -18,6 +18,7 @@
 #include "gemm_pair.cuh"
 #include "quant.cuh"
 #include "attention.cuh"
+#include "gemv.cuh"
 
 namespace {
 
@@ -389,27 +390,54 @@ mxq_status launch_gemm_pairs(mxq_format f, int dev, int sms, int64_t M, int64_t 
                              int64_t ldy, const Epilogue& ep, cudaStream_t s) {
   // slots 6-11: plain epilogue; 12-17: producer epilogue
   const int base = EPI ? 12 : 6;
+  // 256-column tiles, unless they would leave more than half of the CTA pairs
+  // without a tile (e.g. M = 512, N = 3072: 24 tiles for 74 pairs); 128-column
+  // tiles double the count
+  const int64_t tiles256 = ((M + 255) / 256) * ((N + 255) / 256);
+  const bool wide = N > 128 && tiles256 > (sms / 2) / 2;
   switch (f) {
     case MXQ_NVFP4:
-      if (N > 128)
+      if (wide)
         return launch_gemm_pair<mxq::Fmt::NVFP4, 256, EPI>(dev, sms, base, M, N, K, a, a_sf, a_g, b,
                                                            b_sf, b_g, bias, y, ldy, ep, s);
       return launch_gemm_pair<mxq::Fmt::NVFP4, 128, EPI>(dev, sms, base + 1, M, N, K, a, a_sf, a_g, b,
                                                          b_sf, b_g, bias, y, ldy, ep, s);
     case MXQ_MXFP8:
-      if (N > 128)
+      if (wide)
         return launch_gemm_pair<mxq::Fmt::MXFP8, 256, EPI>(dev, sms, base + 2, M, N, K, a, a_sf, a_g, b,
                                                            b_sf, b_g, bias, y, ldy, ep, s);
       return launch_gemm_pair<mxq::Fmt::MXFP8, 128, EPI>(dev, sms, base + 3, M, N, K, a, a_sf, a_g, b,
                                                          b_sf, b_g, bias, y, ldy, ep, s);
     case MXQ_BF16:
-      if (N > 128)
+      if (wide)
         return launch_gemm_pair<mxq::Fmt::BF16, 256, EPI>(dev, sms, base + 4, M, N, K, a, a_sf, a_g, b,
                                                           b_sf, b_g, bias, y, ldy, ep, s);
       return launch_gemm_pair<mxq::Fmt::BF16, 128, EPI>(dev, sms, base + 5, M, N, K, a, a_sf, a_g, b,
                                                         b_sf, b_g, bias, y, ldy, ep, s);
   }
   return MXQ_ERR_INVALID_ARG;
+}
+
+// bf16 layers with M <= 8: CUDA-core weight stream over all SMs (gemv.cuh).
+mxq_status launch_gemv(int sms, int64_t M, int64_t N, int64_t K, const void* x, const void* w,
+                       const void* bias, void* y, int64_t ldy, cudaStream_t s) {
+  const int rw = M <= 2 ? mxq::gemv_rows<2>() : mxq::gemv_rows<8>();
+  const int64_t tasks = (N + rw - 1) / rw;  // one warp each
+  int64_t grid = (tasks + mxq::kGemvThreads / 32 - 1) / (mxq::kGemvThreads / 32);
+  if (grid > static_cast<int64_t>(sms) * 8) grid = static_cast<int64_t>(sms) * 8;
+  if (grid < 1) grid = 1;
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  const auto* wb = static_cast<const __nv_bfloat16*>(w);
+  const auto* bb = static_cast<const __nv_bfloat16*>(bias);
+  auto* yb = static_cast<__nv_bfloat16*>(y);
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  cudaError_t e;
+  const dim3 g(static_cast<unsigned>(grid)), b(mxq::kGemvThreads);
+  if (M == 1) e = launch_pdl(mxq::gemv_bf16_kernel<1>, g, b, 0, s, xb, m, k, wb, n, bb, yb, ldy);
+  else if (M == 2) e = launch_pdl(mxq::gemv_bf16_kernel<2>, g, b, 0, s, xb, m, k, wb, n, bb, yb, ldy);
+  else if (M <= 4) e = launch_pdl(mxq::gemv_bf16_kernel<4>, g, b, 0, s, xb, m, k, wb, n, bb, yb, ldy);
+  else e = launch_pdl(mxq::gemv_bf16_kernel<8>, g, b, 0, s, xb, m, k, wb, n, bb, yb, ldy);
+  return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
 }
 
 mxq_status launch_gemm(mxq_format f, int dev, int sms, int64_t M, int64_t N, int64_t K,
@@ -438,6 +466,7 @@ mxq_status launch_gemm(mxq_format f, int dev, int sms, int64_t M, int64_t N, int
       return launch_gemm_bn<mxq::Fmt::MXFP8, 128>(dev, sms, 3, M, N, K, a, a_sf, a_g, b, b_sf,
                                                    b_g, bias, y, ldy, s);
     case MXQ_BF16:
+      if (M <= mxq::kGemvMaxM) return launch_gemv(sms, M, N, K, a, b, bias, y, ldy, s);
       if (N % 256 == 0)
         return launch_gemm_bn<mxq::Fmt::BF16, 256>(dev, sms, 4, M, N, K, a, a_sf, a_g, b, b_sf,
                                                     b_g, bias, y, ldy, s);

@@ -100,6 +100,28 @@ def test_tolerance_rule():
     assert not bad.any()
 
 
+def test_bf16_rounding_matches_hand_worked_ties_and_torch():
+    # ties to the even significand, by hand: 1 + 2^-8 lies halfway between 1
+    # and 1 + 2^-7 (odd) -> 1; 1 + 3 * 2^-8 halfway between 1 + 2^-7 (odd) and
+    # 1 + 2^-6 (even) -> 1 + 2^-6; the sign is kept; 2^-9 above 1.5 rounds down
+    x = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8), 1.5 + 2.0 ** -9, 0.0, 3.0])
+    assert np.array_equal(G.bf16_rne(x), [1.0, 1 + 2.0 ** -6, -1.0, 1.5, 0.0, 3.0])
+    # float32 inputs: the same as torch's float32 -> bf16 cast (a library routine)
+    rng = np.random.default_rng(3)
+    f = (rng.standard_normal(100000) * np.exp2(rng.integers(-30, 30, 100000))).astype(np.float32)
+    assert np.array_equal(G.bf16_rne(f.astype(np.float64)), torch.tensor(f).bfloat16().double().numpy())
+
+
+def test_correctly_rounded_output_passes_and_one_ulp_off_does_not():
+    # |Y| comparable to T: the bf16 rounding of Y exceeds 2e-3 T
+    Y = np.array([[-0.5408780856523663]])
+    T = np.array([[0.8773537517990917]])
+    good = G.bf16_rne(Y)
+    assert good[0, 0] == -0.5390625 and abs(good[0, 0] - Y[0, 0]) > 2e-3 * T[0, 0] + 1e-6
+    assert G.within_tol(good, Y, T).all()
+    assert not G.within_tol(good - 2.0 ** -8, Y, T).any()
+
+
 def test_quantization_error_within_gemm_tolerance_is_not_vacuous():
     # the bf16 product of the raw operands differs from the quantised one by
     # far more than the tolerance: the tolerance pins the quantised operands
