@@ -25,7 +25,8 @@ from a CUDA graph) against the same stack in bf16 through cuBLAS; use a small
 --steps there (one pass is ~17 ms at batch 1).  --workload attn times the
 8-bit attention (24 heads x 4608 tokens x 128) against bf16 SDPA;
 --workload bf16 times the dispatcher's bf16 branch against torch.addmm on
-the stack's bf16 layers.
+the stack's bf16 layers; --workload mlp4 times the NVFP4 MLP pair at
+M = 16896 with the producer-fed amax (GELU epilogue + max|y|) and without.
 
 --impl reference times the CPU oracle (the plain numpy restatement of the
 method) on a bounded sample of the same workload on the host cores.
@@ -772,6 +773,140 @@ def run_bf16_branch(args, rank, world, local_rank):
     }
 
 
+def run_mlp(args, rank, world, local_rank):
+    """One step = the NVFP4 MLP pair of a single-stream block at 2048 x 2048
+    (M = 16896 tokens): mlp_up 3072 -> 12288 whose epilogue applies GELU, then
+    mlp_down 12288 -> 3072 (the C4 layer) on that output, both through
+    mxq_linear with their activation quantisation.  Timed two ways on the same
+    buffers: producer-fed (mlp_up's epilogue also folds max |y| of its bf16
+    output into one device word, and mlp_down's quantiser takes it instead of
+    its own amax pass: one read of the 415 MB activation) and unfused (mlp_down
+    takes its own amax: two reads).  The GEMMs' own durations come from event
+    pairs mxq_linear records around them; the rest of the step is the two
+    activation quantisations.  Seeded inputs: x ~ N(0, 1), weights ~ N(0,
+    0.02) / N(0, 0.01), biases ~ N(0, 0.02)."""
+    import fp8_gemm_diffusion_b200 as mxq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    M, H, F = 16896, 3072, 12288
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    x = torch.randn(M, H, generator=g, device=dev).to(torch.bfloat16)
+    W1 = (torch.randn(F, H, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    b1 = (torch.randn(F, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    W2 = (torch.randn(H, F, generator=g, device=dev) * 0.01).to(torch.bfloat16)
+    b2 = (torch.randn(H, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    w1 = mxq.Weight(W1, b1, fmt="nvfp4")
+    w2 = mxq.Weight(W2, b2, fmt="nvfp4")
+    del W1, W2
+    h = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(M, H, dtype=torch.bfloat16, device=dev)
+    ws1_bytes = mxq.linear_workspace_bytes(M, H, mxq.NVFP4)
+    ws2_bytes = mxq.linear_workspace_bytes(M, F, mxq.NVFP4)
+    ws1 = torch.empty(ws1_bytes, dtype=torch.uint8, device=dev)
+    ws2 = torch.empty(ws2_bytes, dtype=torch.uint8, device=dev)
+    h_amax = torch.zeros(1, dtype=torch.float32, device=dev)
+    flops = 2.0 * M * H * F * 2
+    launches = {True: mxq.linear_kernel_count(w1.handle, M) + mxq.linear_kernel_count(w2.handle, M, x_amax=h_amax),
+                False: mxq.linear_kernel_count(w1.handle, M) + mxq.linear_kernel_count(w2.handle, M)}
+
+    def step(fused, ev=None):
+        e1 = ev[0] if ev else None
+        e2 = ev[1] if ev else None
+        mxq.linear(w1.handle, x, M, h, ws1, ws1_bytes, stream=stream, gemm_events=e1,
+                   activation=mxq.ACT_GELU, y_amax=h_amax if fused else None)
+        mxq.linear(w2.handle, h, M, y, ws2, ws2_bytes, stream=stream, gemm_events=e2,
+                   x_amax=h_amax if fused else None)
+
+    def timed(fn, n):
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.barrier()
+        torch.cuda.synchronize()
+        torch.cuda._sleep(SPIN_CYCLES)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), dev)
+
+    res = {}
+    sampler = ClockSampler(_nvml_id(local_rank))
+    sampler.start()
+    for fused in (True, False):
+        for _ in range(args.warmup):
+            step(fused)
+        torch.cuda.synchronize()
+        if mxq.get_device_error() != mxq.OK:
+            raise RuntimeError("device-side timeout during warm-up")
+        t0 = time.perf_counter()
+        ms = timed(lambda i: step(fused), args.steps) / args.steps
+        sampler.mark("fused" if fused else "unfused", t0, time.perf_counter())
+        evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
+               for _ in range(args.steps)]
+        for ev in evs:
+            for a, b in ev:
+                a.record(stream)
+                b.record(stream)
+        torch.cuda.synchronize()
+        timed(lambda i: step(fused, evs[i]), args.steps)
+        g1 = float(np.mean([ev[0][0].elapsed_time(ev[0][1]) for ev in evs]))
+        g2 = float(np.mean([ev[1][0].elapsed_time(ev[1][1]) for ev in evs]))
+        if mxq.get_device_error() != mxq.OK:
+            raise RuntimeError("device-side timeout in the timed steps")
+        res[fused] = dict(ms=ms, gemm_up_ms=g1, gemm_down_ms=g2)
+    sampler.stop()
+    fz, un = res[True], res[False]
+    value = whole_job_tflops(world, 1, flops, fz["ms"])
+    peaks = _peaks()
+    peak = peaks["bf16"] * NOMINAL_RATIO["nvfp4"]
+
+    def quant_share(r):
+        q = max(0.0, r["ms"] - r["gemm_up_ms"] - r["gemm_down_ms"])
+        return round(q * 1e3, 2), round(q / r["ms"], 4)
+
+    return {
+        "metric": "NVFP4 MLP-pair TFLOPS incl. activation quantisation (2 x 2MKN per step)",
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(fz["ms"], 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 + e4m3 block scales + fp32 tensor scale); fp32 accumulate; bf16 out",
+        "data": "synthetic (seeded; random-init weights)",
+        "config": {"workload": "mlp_pair_16896x3072x12288_gelu", "M": M, "hidden": H, "mlp": F,
+                   "parallelism": f"replicas x{world}",
+                   "step": "mlp_up (GELU epilogue, max|y| folded into one word) -> mlp_down quantised with "
+                           "that amax (one pass over its 415 MB input) -> GEMM",
+                   "l2": "every buffer of a step (> 1 GB) is larger than L2"},
+        "producer_fed": {"ms_per_step": round(fz["ms"], 5), "gemm_up_us": round(fz["gemm_up_ms"] * 1e3, 2),
+                         "gemm_down_us": round(fz["gemm_down_ms"] * 1e3, 2),
+                         "quantisation_us": quant_share(fz)[0], "quantisation_share": quant_share(fz)[1]},
+        "unfused": {"ms_per_step": round(un["ms"], 5), "value": round(whole_job_tflops(world, 1, flops, un["ms"]), 2),
+                    "gemm_up_us": round(un["gemm_up_ms"] * 1e3, 2), "gemm_down_us": round(un["gemm_down_ms"] * 1e3, 2),
+                    "quantisation_us": quant_share(un)[0], "quantisation_share": quant_share(un)[1]},
+        "speedup_of_fusion": round(un["ms"] / fz["ms"], 4),
+        "roofline": {"kernel": "gemm_pair_kernel<NVFP4> x 2 + quantisers", "bound": "tensor",
+                     "achieved": round(value, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                     "frac": round(value / peak, 4), "peak_kind": "burst",
+                     "peak_source": f"{peaks['source']} bf16 burst x 4 (nvfp4 dense ratio); whole step",
+                     "traffic": None},
+        "clocks": sampler.summary("fused"),
+        "e2e": None,
+        "gpu_launches": launches[True] * args.steps,
+        "cpu_baseline": None,
+    }
+
+
 # ------------------------------------------------------------- attention
 def run_attention(args, rank, world, local_rank):
     """One step = one FLUX-shaped attention (24 heads x 4608 tokens x 128)
@@ -939,7 +1074,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5", "attn", "bf16"])
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5", "attn", "bf16", "mlp4"])
     ap.add_argument("--batch", type=int, default=1, choices=[1, 4],
                     help="batch of the c5 stack (1: 4608 tokens per image)")
     ap.add_argument("--impl", default="mxq", choices=["mxq", "reference"])
@@ -962,7 +1097,7 @@ def main():
         # the CPU oracle on the host cores: rank 0 only, a few bounded samples
         if rank != 0:
             return 0
-        if args.workload in ("c5", "attn", "bf16"):
+        if args.workload in ("c5", "attn", "bf16", "mlp4"):
             print(json.dumps({"impl": "reference", "unavailable": "the oracle arm times single "
                               "linear layers (c1-c4)"}))
             return 0
@@ -994,8 +1129,8 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device("cuda", local_rank))
     try:
-        if args.workload in ("c5", "attn", "bf16"):
-            fn = {"c5": run_stack, "attn": run_attention, "bf16": run_bf16_branch}[args.workload]
+        if args.workload in ("c5", "attn", "bf16", "mlp4"):
+            fn = {"c5": run_stack, "attn": run_attention, "bf16": run_bf16_branch, "mlp4": run_mlp}[args.workload]
             result = fn(args, rank, world, local_rank)
             if rank == 0:
                 print(json.dumps(result))

@@ -106,12 +106,6 @@ struct AttArgs {
   __nv_bfloat16* out;               // [heads][tokens][128]
 };
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // MXFP8 shared exponent by the ceiling rule for a block maximum that is 0
 // or a normal fp32: the smallest X with bmax <= 448 * 2^X, clamped to
 // [-127, 127].  With bmax = (1 + f) 2^e, 448 * 2^(e - 8) = 1.75 * 2^e, so X is

@@ -163,9 +163,24 @@ struct PairArgs {
   unsigned int* y_amax;   // EPI != 0 only: max |y| over the bf16 outputs, folded in with atomicMax
 };
 
-// GELU with the exact error function, x * Phi(x), in fp32.
+// GELU, x * Phi(x), Phi(x) = (1 + erf(x / sqrt 2)) / 2, in fp32, with erf by
+// formula 7.1.26 of Abramowitz and Stegun's Handbook of Mathematical
+// Functions: for z >= 0, 1 - erf(z) = t (a1 + t (a2 + t (a3 + t (a4 + t a5))))
+// e^(-z^2), t = 1 / (1 + p z), absolute error at most 1.5e-7.  With
+// z = |x| / sqrt 2 and q = 1 - erf(z): GELU(x) = x - x q / 2 for x >= 0 and
+// x q / 2 for x < 0 (no cancellation on the negative side).  Two
+// special-function operations (the reciprocal and 2^x) and a dozen FMAs: the
+// epilogue of a whole tile then stays within the tile's MMA time.
 __device__ __forceinline__ float gelu_erf(float x) {
-  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+  const float t = rcp_approx(fmaf(0.3275911f * 0.70710678118654752f, fabsf(x), 1.0f));
+  float p = 1.061405429f;
+  p = fmaf(p, t, -1.453152027f);
+  p = fmaf(p, t, 1.421413741f);
+  p = fmaf(p, t, -0.284496736f);
+  p = fmaf(p, t, 0.254829592f);
+  const float e = ex2_approx(-0.72134752044448170f * x * x);  // e^(-x^2 / 2)
+  const float hq = 0.5f * x * (p * t) * e;                      // x q / 2
+  return x >= 0.0f ? x - hq : hq;
 }
 
 // EPI = 0: the plain epilogue.  EPI = 1: the producer epilogue of a layer

@@ -218,7 +218,11 @@ mxq_status mxq_weight_prepare(mxq_format f, const void* w_bf16, int64_t N, int64
                               size_t storage_bytes, mxq_weight* out, mxq_stream_t stream);
 
 /* Activation applied in the GEMM epilogue (mxq_linear_opts.activation). */
-enum { MXQ_ACT_NONE = 0, MXQ_ACT_GELU = 1 /* x * Phi(x), exact erf */ };
+enum {
+  MXQ_ACT_NONE = 0,
+  MXQ_ACT_GELU = 1 /* x * Phi(x) with the error function (not the tanh form); erf evaluated in
+                      fp32 by Abramowitz and Stegun 7.1.26, |error| <= 1.5e-7 */
+};
 
 /* Options of mxq_linear.  A NULL pointer means the defaults; a zeroed struct
  * is the defaults too. */
