@@ -193,6 +193,15 @@ def whole_job_tflops(world: int, steps: int, flops_per_step: float, max_ms: floa
 
 
 # ------------------------------------------------------------ the GPU arm
+def default_min_dim(case_name: str, requested):
+    """min_dim passed to mxq_linear: the caller's, else 1 for C1 (the NVFP4 W4A4
+    single-GEMM configuration, 256 x 1024 x 1024, which the selective rule
+    would otherwise keep in bf16), else the library's default (None)."""
+    if requested is not None:
+        return requested
+    return 1 if case_name.startswith("c1") else None
+
+
 def run_gpu(args, rank, world, local_rank):
     import fp8_gemm_diffusion_b200 as mxq
 
@@ -251,7 +260,7 @@ def run_gpu(args, rank, world, local_rank):
     # single-GEMM configuration: its 256 x 1024 x 1024 shape is below the
     # selective rule's 1024 threshold, so it is run with min_dim = 1 to time
     # the NVFP4 path it names (the line reports the path actually taken).
-    min_dim = args.min_dim if args.min_dim is not None else (1 if case.name.startswith("c1") else None)
+    min_dim = default_min_dim(case.name, args.min_dim)
     path = mxq.linear_path(base_w.handle, M, min_dim)
     run_fmt = {mxq.NVFP4: "nvfp4", mxq.MXFP8: "mxfp8", mxq.BF16: "bf16"}[path]
 

@@ -535,9 +535,11 @@ __global__ void __launch_bounds__(kMxThreads)
        t += static_cast<int64_t>(gridDim.x) * kMxThreads) {
     const int r = static_cast<int>(t / bpr), c = static_cast<int>(t - static_cast<int64_t>(r) * bpr);
     const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ld + 32 * c);
+    // each 16-byte load covers half of a 32-byte sector per lane; loads that
+    // allocate in L1 serve the other half from there instead of L2
     uint4 u[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) u[i] = ldg_nc_v4(src + i);
+    for (int i = 0; i < 4; ++i) u[i] = ldg_nc_v4_l1(src + i);
     float f[32];
 #pragma unroll
     for (int i = 0; i < 4; ++i) bf16x8_to_f32(u[i], *reinterpret_cast<float(*)[8]>(f + 8 * i));

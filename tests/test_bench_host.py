@@ -71,3 +71,22 @@ def test_peaks_come_from_the_measured_file_or_the_fallback():
     assert p["source"] in ("measured", "fallback")
     assert p["bf16"] > 0 and p["bf16_sustained"] > 0 and p["hbm"] > 0
     assert bench.whole_job_tflops(2, 10, 1e12, 1000.0) == 20.0
+
+
+def test_c1_line_takes_the_nvfp4_path_it_names():
+    # C1 (NVFP4 W4A4, 256 x 1024 x 1024) is below the selective rule's 1024:
+    # the bench passes min_dim = 1 so that the step runs (and the line
+    # reports) the NVFP4 path; mxq_linear_path is host logic on the weight
+    # descriptor, so no device is needed
+    import bench
+    import workloads
+
+    import fp8_gemm_diffusion_b200 as mxq
+
+    name = workloads.CASE_NAMES["c1"]
+    w = mxq.mxq_weight(format=mxq.NVFP4, flags=0, N=1024, K=1024)
+    assert bench.default_min_dim(name, None) == 1
+    assert mxq.linear_path(w, 256, bench.default_min_dim(name, None)) == mxq.NVFP4
+    assert mxq.linear_path(w, 256, None) == mxq.BF16  # the library default keeps it in bf16
+    assert bench.default_min_dim(workloads.CASE_NAMES["c3"], None) is None
+    assert bench.default_min_dim(name, 4096) == 4096
