@@ -67,7 +67,7 @@ NOMINAL_RATIO = {"nvfp4": 4.0, "mxfp8": 2.0, "bf16": 1.0}
 # DRAM bytes (read + write) of one launch of the roofline's kernel, from one
 # ncu capture of the committed kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum); None where no capture of the current kernel exists.
-GEMM_TRAFFIC_BYTES = {"c3_nvfp4_4608x3072x12288": 92455680}
+GEMM_TRAFFIC_BYTES = {"c3_nvfp4_4608x3072x12288": 92199680}
 
 
 def _peaks():
@@ -417,6 +417,10 @@ def run_gpu(args, rank, world, local_rank):
             "quantize_public_calls": round(quant_pub_ms, 5),
         },
         "quantize_gbs": round(qbytes / (max(step_ms - gemm_ms, 1e-6) * 1e-3) / 1e9, 1),
+        "quantize_note": "algorithmic bytes over quantize_in_step = the step (launches overlapping through "
+                         "programmatic dependent launch) minus the GEMM timed with events around it (which "
+                         "costs it that overlap): the quantiser's share of the step, not its standalone "
+                         "duration (quantize_public_calls times the public calls alone, launch gaps included)",
         "hot": {"value": round(whole_job_tflops(world, 1, flops, hot_ms), 2), "unit": UNIT,
                 "ms_per_step": round(hot_ms, 5), "steps": hot_steps,
                 "l2": "one buffer set reused every step (inputs L2-resident)"},
