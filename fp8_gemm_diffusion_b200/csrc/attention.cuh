@@ -523,27 +523,26 @@ __global__ void __launch_bounds__(kVtThreads) quantize_mxfp8_vt_kernel(const __n
     stile[threadIdx.x + i * kVtThreads] = ldg_nc_v4(src + threadIdx.x + i * kVtThreads);
   __syncthreads();
   const int p = threadIdx.x & 63, blk = threadIdx.x >> 6;
-  float f0[32], f1[32];
+  // the two channels' 32 values stay packed as bf16 pairs (32 registers)
+  uint32_t pr[32];
   float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&tile[32 * blk + i][2 * p]);
-    f0[i] = __low2float(pr);
-    f1[i] = __high2float(pr);
-    m0 = fmaxf(m0, fabsf(f0[i]));
-    m1 = fmaxf(m1, fabsf(f1[i]));
+    pr[i] = *reinterpret_cast<const uint32_t*>(&tile[32 * blk + i][2 * p]);
+    m0 = fmaxf(m0, fabsf(__uint_as_float(pr[i] << 16)));
+    m1 = fmaxf(m1, fabsf(__uint_as_float(pr[i] & 0xFFFF0000u)));
   }
 #pragma unroll
   for (int ch = 0; ch < 2; ++ch) {
-    const float* f = ch == 0 ? f0 : f1;
     const float bmax = ch == 0 ? m0 : m1;
     int X = -127;
     if (bmax > 0.0f) X = min(max(floor_log2_f32(bmax) - 8, -127), 127);  // OCP floor rule
     const float mult = exp2_int(-X);
+    auto val = [&](int i) { return __uint_as_float(ch == 0 ? pr[i] << 16 : pr[i] & 0xFFFF0000u) * mult; };
     uint32_t w[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      w[i] = cvt_e4m3x2(f[4 * i] * mult, f[4 * i + 1] * mult) | (cvt_e4m3x2(f[4 * i + 2] * mult, f[4 * i + 3] * mult) << 16);
+      w[i] = cvt_e4m3x2(val(4 * i), val(4 * i + 1)) | (cvt_e4m3x2(val(4 * i + 2), val(4 * i + 3)) << 16);
     const int64_t row = static_cast<int64_t>(h) * kAttD + 2 * p + ch;
     uint4* dst = reinterpret_cast<uint4*>(codes + row * tokens + t0 + 32 * blk);
     dst[0] = make_uint4(w[0], w[1], w[2], w[3]);

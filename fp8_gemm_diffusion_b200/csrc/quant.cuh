@@ -270,7 +270,11 @@ __global__ void __launch_bounds__(kQuantThreads)
   const int warps = gridDim.x * (kQuantThreads / 32);
   const int bpr = k >> 4;  // 16-element blocks per row, one per lane per step
   const uint32_t c4 = static_cast<uint32_t>(k >> 6);  // 4-column scale groups per row
-  for (int r = blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
+  // rows last to first: the amax pass just before read them first to last,
+  // so the tail of the activation is still in L2 when this pass starts, and
+  // the rows this pass writes last (the first ones) are where the GEMM begins
+  for (int rr = blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5); rr < rows; rr += warps) {
+    const int r = rows - 1 - rr;
     const __nv_bfloat16* row = x + static_cast<int64_t>(r) * ld;
     uint2* crow = reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * (k >> 1));
     // this row's scale bytes: 512-byte tile (r / 128, c / 4), byte (r % 32) * 16 + (r / 32 % 4) * 4 + c % 4
