@@ -140,6 +140,20 @@ class ClockSampler:
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
 
+    def sample_until(self, event, max_s: float = 5.0):
+        """Sample from the calling thread until `event` has completed: the
+        timed region's last milliseconds, after the host has enqueued its
+        work, while the sampler thread may still be waiting for the
+        interpreter lock."""
+        if self._h is None:
+            return
+        t0 = time.perf_counter()
+        while not event.query() and time.perf_counter() - t0 < max_s:
+            try:
+                self._sample()
+            except Exception:
+                return
+
     def mark(self, name, t0, t1):
         """Record [t0, t1] (host perf_counter times) as a named window."""
         self.windows[name] = (t0, t1)
@@ -315,6 +329,7 @@ def run_gpu(args, rank, world, local_rank):
         for i in range(n):
             fn(i)
         t_end.record(stream)
+        sampler.sample_until(t_end)
         torch.cuda.synchronize()
         sampler.mark(name, h0, time.perf_counter())
         if dist:

@@ -59,6 +59,36 @@ def test_clock_summary_flags_throttling_and_counts_windows():
     assert s.summary()["reasons"] == ["unavailable"]
 
 
+def test_samples_are_taken_until_the_timed_region_ends():
+    # the main thread samples while the last steps run (a fake event that
+    # completes on its fourth query, a fake NVML)
+    class Ev:
+        n = 0
+
+        def query(self):
+            Ev.n += 1
+            return Ev.n > 3
+
+    class NV:
+        NVML_CLOCK_SM = 0
+
+        @staticmethod
+        def nvmlDeviceGetClockInfo(h, which):
+            return 1965
+
+        @staticmethod
+        def nvmlDeviceGetCurrentClocksEventReasons(h):
+            return 0x4
+
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s._h, s._nv, s.samples = object(), NV, []
+    s.sample_until(Ev())
+    assert len(s.samples) == 3 and all(m == 1965 and r == 0x4 for _, m, r in s.samples)
+    s._h = None
+    s.sample_until(Ev())  # no NVML: nothing, no error
+    assert len(s.samples) == 3
+
+
 def test_sustained_peak_needs_a_long_timed_region():
     # the denominator switches to the sustained figure only for a GEMM timed
     # inside a region of at least a second
