@@ -212,7 +212,7 @@ FusedPlan plan_fused(int64_t rows, int64_t k, int sms) {
 }
 
 // Cooperative launch (the grid barrier needs every CTA resident), with
-// programmatic stream serialization when the driver accepts both.
+// programmatic stream serialization when the CUDA driver accepts both.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_coop(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                         Args... args) {
