@@ -40,9 +40,9 @@
 //               exponential unit busy).  Per block:
 //               block maxima, the normaliser (taken over from the other
 //               warpgroup's previous block through shared memory and raised
-//               if needed), weights, MXFP8 codes of E into shared memory
-//               (the second product's A operand) and their scales into
-//               tensor memory; at the end O / rowsum -> bf16.
+//               if needed), weights, MXFP8 codes of E and their scales
+//               into tensor memory (the second product's A operand); at
+//               the end O / rowsum -> bf16.
 // Every wait is bounded (ptx.cuh).  The softmax warps never leave their
 // loop early: after a timeout they skip the work but keep the hand-over
 // order, so no warp waits on a named barrier that is never signalled.
@@ -72,8 +72,7 @@ struct AttCfg {
   static constexpr int OFF_QSF = TILE_BYTES;                        // Q scale chunk (512 B)
   static constexpr int OFF_ONESF = TILE_BYTES + 512;                // unit scales of the extension rows
   static constexpr int OFF_STAGE = TILE_BYTES + 1024;
-  static constexpr int OFF_P = OFF_STAGE + kAttStages * STAGE_BYTES;  // two E-code buffers
-  static constexpr int OFF_XCH = OFF_P + 2 * TILE_BYTES;            // [128 rows] normaliser, [4] flags
+  static constexpr int OFF_XCH = OFF_STAGE + kAttStages * STAGE_BYTES;  // [128 rows] normaliser, [4] flags
   static constexpr int XCH_BYTES = 128 * 4 + 64;
   static constexpr int OFF_BAR = OFF_XCH + XCH_BYTES;
   static constexpr int BAR_BYTES = 256;
@@ -83,9 +82,12 @@ struct AttCfg {
   // 15 zero columns
   static constexpr int PV_N = kAttD + 16;
   // tensor memory columns: two S buffers, O (144), scale columns of Q, K,
-  // V^T (two 128-row groups: the tile's and the extension's), and of the
-  // weights (one 4-column group per S buffer)
-  static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 400, T_KSF = 404, T_VSF = 408, T_PSF = 416;
+  // V^T (two 128-row groups: the tile's and the extension's), of the
+  // weights (one 4-column group per S buffer), then the weights' E4M3 codes
+  // themselves, the second product's A operand (32 columns per S buffer:
+  // four codes per column, the row in the lane)
+  static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 400, T_KSF = 404, T_VSF = 408, T_PSF = 416,
+                            T_P = 424;
   static constexpr int TMEM_COLS = 512;
   static constexpr int THREADS = 384;
   static constexpr int SOFT_WARP0 = 4;
@@ -94,7 +96,8 @@ struct AttCfg {
   static constexpr int REGS_CTRL = 56, REGS_SOFT = 224;
 };
 static_assert(AttCfg::STAGE_BYTES % 1024 == 0, "stage alignment (128-byte swizzle atoms)");
-static_assert(AttCfg::T_PSF + 8 <= AttCfg::TMEM_COLS && AttCfg::T_O + AttCfg::PV_N <= AttCfg::T_QSF, "tensor memory");
+static_assert(AttCfg::T_P + 64 <= AttCfg::TMEM_COLS && AttCfg::T_PSF + 8 <= AttCfg::T_P &&
+                  AttCfg::T_O + AttCfg::PV_N <= AttCfg::T_QSF, "tensor memory");
 static_assert(128 * AttCfg::REGS_CTRL + 256 * AttCfg::REGS_SOFT <= 384 * 168, "register split");
 
 struct AttArgs {
@@ -339,13 +342,12 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
           tc_fence_after();
           const uint32_t st = base + C::OFF_STAGE + st_idx * C::STAGE_BYTES;
           tc_cp_32x128b_warpx4(tmem + C::T_VSF, desc_sf_chunk(st + C::ST_VSF));
-          const uint64_t pdesc = desc_kmajor_sw128(base + C::OFF_P + b * C::TILE_BYTES);
           const uint64_t vdesc = desc_kmajor_sw128(st + C::TILE_BYTES);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             // MMA k covers keys [32 k, 32 k + 32), scale byte k of the row's word
             const uint64_t koff = static_cast<uint64_t>(2 * k);
-            mma_mxfp8(tmem + C::T_O, pdesc + koff, vdesc + koff, idesc_mxfp8_m128(C::PV_N, k, k),
+            mma_mxfp8_ta(tmem + C::T_O, tmem + C::T_P + 32 * b + 8 * k, vdesc + koff, idesc_mxfp8_m128(C::PV_N, k, k),
                       (tmem + C::T_PSF + 4 * b) | (static_cast<uint32_t>(k) << 30),
                       (tmem + C::T_VSF) | (static_cast<uint32_t>(k) << 30), (j > 0 || k > 0) ? 1u : 0u);
           }
@@ -473,17 +475,9 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
       ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(p_free(b), ((j >> 1) & 1) ^ 1u));
       if (ok) {
         tc_fence_after();
-        // row r of the A operand: 128 bytes, 128-byte swizzle (chunk ch at ch ^ (r % 8))
-        const uint32_t prow = base + C::OFF_P + b * C::TILE_BYTES + r * 128;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint32_t addr = prow + ((ch ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(codes[4 * ch]),
-                       "r"(codes[4 * ch + 1]), "r"(codes[4 * ch + 2]), "r"(codes[4 * ch + 3])
-                       : "memory");
-        }
-        fence_proxy_async_smem();
-        // the row's four block scales, on the sub-partition's diagonal column
+        // the row's codes into tensor memory (the second product's A operand)
+        // and its four block scales, on the sub-partition's diagonal column
+        tmem_st_32x32b_x32(trow + C::T_P + 32 * b, codes);
         tmem_st_32x32b_x1(trow + C::T_PSF + 4 * b + q, sfw);
         tc_wait_st();
         tc_fence_before();
