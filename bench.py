@@ -67,7 +67,8 @@ NOMINAL_RATIO = {"nvfp4": 4.0, "mxfp8": 2.0, "bf16": 1.0}
 # DRAM bytes (read + write) of one launch of the roofline's kernel, from one
 # ncu capture of the committed kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum); None where no capture of the current kernel exists.
-GEMM_TRAFFIC_BYTES = {"c3_nvfp4_4608x3072x12288": 92199680}
+GEMM_TRAFFIC_BYTES = {"c3_nvfp4_4608x3072x12288": 92199680, "c2_mxfp8_4608x3072x9216": 87975936,
+                      "c4_nvfp4_16896x12288x3072": 222627840}
 
 
 def _peaks():
