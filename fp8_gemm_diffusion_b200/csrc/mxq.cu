@@ -113,11 +113,13 @@ mxq_status tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uin
   return MXQ_OK;
 }
 
-// One warp per row: enough blocks to give every row a warp, at most 8 blocks
-// per SM and at most kMaxAmaxPartials blocks (the partial-amax array size).
-int quant_grid(int64_t rows, int sms) {
+// Grid of the two-pass kernels, which deal row chunks of `chunk_elems`
+// elements to warps: a warp per chunk up to 8 blocks per SM and at most
+// kMaxAmaxPartials blocks (the partial-amax array size).
+int quant_grid(int64_t rows, int64_t k, int64_t chunk_elems, int sms) {
   const int64_t warps_per_block = mxq::kQuantThreads / 32;
-  int64_t g = (rows + warps_per_block - 1) / warps_per_block;
+  const int64_t chunks = rows * ((k + chunk_elems - 1) / chunk_elems);
+  int64_t g = (chunks + warps_per_block - 1) / warps_per_block;
   int64_t cap = static_cast<int64_t>(sms) * 8;
   if (cap > mxq::kMaxAmaxPartials) cap = mxq::kMaxAmaxPartials;
   if (g > cap) g = cap;
@@ -161,7 +163,7 @@ mxq_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ld, float
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
   if (e != cudaSuccess) return cuda_fail(e);
   if (rows == 0 || k == 0) return MXQ_OK;
-  e = launch_pdl(mxq::amax_kernel, dim3(quant_grid(rows, sms)), dim3(mxq::kQuantThreads), 0, s,
+  e = launch_pdl(mxq::amax_kernel, dim3(quant_grid(rows, k, mxq::kAmaxChunk, sms)), dim3(mxq::kQuantThreads), 0, s,
                  static_cast<const __nv_bfloat16*>(x), static_cast<int>(rows), static_cast<int>(k), ld,
                  static_cast<float*>(nullptr), amax);
   return e == cudaSuccess ? MXQ_OK : cuda_fail(e);
@@ -170,7 +172,7 @@ mxq_status launch_amax(const void* x, int64_t rows, int64_t k, int64_t ld, float
 // amax as per-block partial maxima (no zeroing needed); returns their count.
 mxq_status launch_amax_partials(const void* x, int64_t rows, int64_t k, int64_t ld, float* partials,
                                 int* n_partials, cudaStream_t s, int sms) {
-  const int grid = quant_grid(rows, sms);
+  const int grid = quant_grid(rows, k, mxq::kAmaxChunk, sms);
   cudaError_t e = launch_pdl(mxq::amax_kernel, dim3(grid), dim3(mxq::kQuantThreads), 0, s,
                              static_cast<const __nv_bfloat16*>(x), static_cast<int>(rows),
                              static_cast<int>(k), ld, partials, static_cast<float*>(nullptr));
@@ -181,7 +183,7 @@ mxq_status launch_amax_partials(const void* x, int64_t rows, int64_t k, int64_t 
 mxq_status launch_quant_nvfp4(const void* x, int64_t rows, int64_t k, int64_t ld,
                               const float* amax_vals, int n_amax, uint8_t* codes, uint8_t* sf,
                               float* g, float* amax_out, cudaStream_t s, int sms) {
-  cudaError_t e = launch_pdl(mxq::quantize_nvfp4_kernel, dim3(quant_grid(rows, sms)),
+  cudaError_t e = launch_pdl(mxq::quantize_nvfp4_kernel, dim3(quant_grid(rows, k, mxq::kNvfp4Chunk, sms)),
                              dim3(mxq::kQuantThreads), 0, s, static_cast<const __nv_bfloat16*>(x),
                              static_cast<int>(rows), static_cast<int>(k), ld, amax_vals, n_amax, codes,
                              sf, g, amax_out);

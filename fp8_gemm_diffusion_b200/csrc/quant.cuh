@@ -20,11 +20,12 @@
 // Conversions use the hardware cvt.rn.satfinite instructions (RNE, finite
 // overflow saturates to the largest magnitude, sign kept).
 //
-// Memory layout: one warp per row.  NVFP4: one lane per 16-element block
-// (two 16-byte loads), so the block's scale arithmetic runs once per block;
-// MXFP8: one 16-byte vector per lane, the 4 lanes of a 32-element block
-// combine their maxima with warp shuffles.  Scale bytes go straight to the
-// tensor-core block-scaling layout (see sf_offset).
+// Work split: the amax and NVFP4 passes deal fixed-size row chunks to warps
+// (ChunkWalk); NVFP4 encodes one 16-element block per lane (two 16-byte
+// loads), so the block's scale arithmetic runs once per block.  MXFP8: one
+// thread per 32-element block, consecutive threads on consecutive blocks.
+// Scale bytes go straight to the tensor-core block-scaling layout (see
+// sf_offset).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -143,11 +144,12 @@ __device__ __forceinline__ void bf16x16_to_f32(const uint4& u0, const uint4& u1,
 }
 
 // ------------------------------------------------------------------- amax
-// Work split: one warp per row (rows strided over all warps of the grid); a
-// lane owns every 32nd 16-byte vector of the row, four loads in flight.  No
-// integer division anywhere on the path.
+// A warp's chunk is 32 x kQuantUnroll consecutive 16-byte vectors of a row:
+// lane l loads vectors l, l + 32, ..., four loads in flight.
 constexpr int kQuantThreads = 256;
 constexpr int kQuantUnroll = 4;
+constexpr int kAmaxChunk = 32 * kQuantUnroll * 8;    // elements per chunk of the amax pass
+constexpr int kNvfp4Chunk = 32 * kQuantUnroll * 16;  // elements per chunk of the NVFP4 pass
 constexpr int kMaxAmaxPartials = 1024;
 
 __device__ __forceinline__ float warp_max(float m) {
@@ -169,7 +171,35 @@ __device__ __forceinline__ float block_max(float m) {
   return b;
 }
 
-// max |x| of the rows this block's warps own, written to partial[blockIdx.x]
+// Work split of the two-pass kernels: each row is cut into chunks of a fixed
+// number of vectors (32 lanes x kQuantUnroll), and the chunks of all rows are
+// dealt to the warps in turn, so every warp gets the same share to within one
+// chunk.  (With whole rows per warp, 16896 rows on 8192 warps left a third
+// round of rows to 512 warps, which could not keep HBM busy: ~12 us of the
+// amax pass's 73 us.)  The walk advances (row, chunk) by the grid's warp count
+// without a division per step.
+// (Rows are below 2^31 and a step adds at most the grid's warp count, 8192,
+// to the row, so the unsigned row never wraps before it passes the last row.)
+struct ChunkWalk {
+  unsigned int r;    // row
+  unsigned int c;    // chunk within the row
+  unsigned int dr;   // rows per step
+  unsigned int dc;   // chunks per step beyond whole rows
+  unsigned int cpr;  // chunks per row
+  __device__ __forceinline__ ChunkWalk(unsigned int first, unsigned int step, unsigned int chunks_per_row)
+      : r(first / chunks_per_row), c(first % chunks_per_row), dr(step / chunks_per_row),
+        dc(step % chunks_per_row), cpr(chunks_per_row) {}
+  __device__ __forceinline__ void next() {
+    r += dr;
+    c += dc;
+    if (c >= cpr) {
+      c -= cpr;
+      ++r;
+    }
+  }
+};
+
+// max |x| of the chunks this block's warps own, written to partial[blockIdx.x]
 // (or folded into *amax_atomic with atomicMax when partial is null).
 __global__ void __launch_bounds__(kQuantThreads) amax_kernel(const __nv_bfloat16* __restrict__ x,
                                                              int rows, int k, int64_t ld,
@@ -180,10 +210,13 @@ __global__ void __launch_bounds__(kQuantThreads) amax_kernel(const __nv_bfloat16
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (kQuantThreads / 32);
   const int vpr = k >> 3;  // 16-byte vectors per row
+  const int cpr = (vpr + 32 * kQuantUnroll - 1) / (32 * kQuantUnroll);  // chunks per row
   float m = 0.0f;
-  for (int r = blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
-    const __nv_bfloat16* row = x + static_cast<int64_t>(r) * ld;
-    for (int v0 = lane; v0 < vpr; v0 += 32 * kQuantUnroll) {
+  if (cpr > 0) {
+    for (ChunkWalk w(blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5), warps, cpr);
+         w.r < static_cast<unsigned int>(rows); w.next()) {
+      const __nv_bfloat16* row = x + static_cast<int64_t>(w.r) * ld;
+      const int v0 = static_cast<int>(w.c) * (32 * kQuantUnroll) + lane;
       uint4 u[kQuantUnroll];
 #pragma unroll
       for (int j = 0; j < kQuantUnroll; ++j) {
@@ -250,7 +283,7 @@ constexpr unsigned long long kKeyMask = 0xFFFFFFFF00000000ull;
 
 // amax_in: n_amax values whose max is the tensor's amax (1 value, or the
 // per-block partials of amax_kernel).
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, 4)
     quantize_nvfp4_kernel(const __nv_bfloat16* __restrict__ x, int rows, int k, int64_t ld,
                           const float* __restrict__ amax_in, int n_amax, uint8_t* __restrict__ codes,
                           uint8_t* __restrict__ sf, float* __restrict__ g_out,
@@ -269,17 +302,20 @@ __global__ void __launch_bounds__(kQuantThreads)
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (kQuantThreads / 32);
   const int bpr = k >> 4;  // 16-element blocks per row, one per lane per step
+  const int cpr = (bpr + 32 * kQuantUnroll - 1) / (32 * kQuantUnroll);  // chunks per row
   const uint32_t c4 = static_cast<uint32_t>(k >> 6);  // 4-column scale groups per row
   // rows last to first: the amax pass just before read them first to last,
   // so the tail of the activation is still in L2 when this pass starts, and
   // the rows this pass writes last (the first ones) are where the GEMM begins
-  for (int rr = blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5); rr < rows; rr += warps) {
-    const int r = rows - 1 - rr;
-    const __nv_bfloat16* row = x + static_cast<int64_t>(r) * ld;
-    uint2* crow = reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * (k >> 1));
-    // this row's scale bytes: 512-byte tile (r / 128, c / 4), byte (r % 32) * 16 + (r / 32 % 4) * 4 + c % 4
-    uint8_t* sf_row = sf + static_cast<int64_t>(r >> 7) * c4 * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
-    for (int c0 = lane; c0 < bpr; c0 += 32 * kQuantUnroll) {
+  if (cpr > 0) {
+    for (ChunkWalk w(blockIdx.x * (kQuantThreads / 32) + (threadIdx.x >> 5), warps, cpr);
+         w.r < static_cast<unsigned int>(rows); w.next()) {
+      const int r = rows - 1 - static_cast<int>(w.r);
+      const __nv_bfloat16* row = x + static_cast<int64_t>(r) * ld;
+      uint2* crow = reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * (k >> 1));
+      // this row's scale bytes: 512-byte tile (r / 128, c / 4), byte (r % 32) * 16 + (r / 32 % 4) * 4 + c % 4
+      uint8_t* sf_row = sf + static_cast<int64_t>(r >> 7) * c4 * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
+      const int c0 = static_cast<int>(w.c) * (32 * kQuantUnroll) + lane;
       uint4 u[kQuantUnroll][2];
 #pragma unroll
       for (int j = 0; j < kQuantUnroll; ++j) {
