@@ -65,6 +65,11 @@ NVFP4_CASES = [
     ("rows77_k192", lambda: workloads.random_case(77, 192, 8, "nvfp4", seed=2).A),
     ("rows130_k320", lambda: workloads.random_case(130, 320, 8, "nvfp4", seed=3).A),
     ("rows257_k1024", lambda: workloads.random_case(257, 1024, 8, "nvfp4", seed=4, a_std=1e-3).A),
+    # the two-pass kernels deal row chunks to warps (1024 elements for the
+    # amax, 2048 for the encode pass): K = 5184 ends both on a partial chunk,
+    # and 3000 rows give more chunks than warps, so a warp's walk carries
+    # from one row's chunks into the next row's
+    ("rows3000_k5184", lambda: workloads.random_case(3000, 5184, 8, "nvfp4", seed=7).A),
 ]
 
 
