@@ -1109,8 +1109,9 @@ class OracleArm:
             "cores": threads,
             "kind": "oracle",
             "sample": f"{steps} step(s) over {rows} rows of {case.name} ({case.M} rows, wrapping "
-                      f"around): {self.chunk}-row chunks, each its amax (nvfp4), {self.fmt} "
-                      f"quantisation and float64 GEMM (Y and sum|ab|); {dt:.1f} s timed",
+                      f"around): {self.chunk}-row chunks, each "
+                      f"{'its amax, ' if self.fmt == 'nvfp4' else ''}{self.fmt} quantisation and "
+                      f"float64 GEMM (Y and sum|ab|); {dt:.1f} s timed",
         }
 
 
