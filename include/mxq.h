@@ -289,7 +289,7 @@ mxq_status mxq_linear(const mxq_weight* w, const void* x_bf16, int64_t M, void* 
  * memory: for example a host whose device-memory budget is fixed at start-up
  * and that forbids allocations afterwards, or a latency-critical loop where
  * cudaMalloc (it may synchronise the device and its latency is unbounded) is
- * not acceptable.  The paper has no counterpart: it is an addition of this
+ * not acceptable.  The method has no such call: it is an addition of this
  * library.
  * Same arguments and result as mxq_linear, without ws / ws_bytes: the
  * workspace for the quantised activation lives in a file-scope device array of
